@@ -1,0 +1,175 @@
+/*
+ * lbq.h -- C ABI of the low-bit weight-only GEMV/GEMM library for B200 (sm_100a).
+ *
+ * The library computes y = s * T(W)^T * (H x): bf16 activations times LLM weights
+ * stored in one of three packed low-bit formats, dequantized on the fly inside
+ * the kernels, accumulated in fp32 and written as bf16.
+ *
+ * Sources (web pages on extreme low-bit 27B inference):
+ *   [tern]  pptc.cn, "8 GB card runs a ternary 27B" article: §1.2 (three states,
+ *           log2 3 bits per weight; products become add / subtract / skip), §5.1
+ *           (absmean ternarisation: s = mean|w|, t = clip(round(w/s), -1, 1)).
+ *   [block] mhpq.cn, "27B in 5.9 GB" article: §2.1 (one shared scale per block of
+ *           64 or 128 weights, weight = trit * scale), §2.2 (ternary matmul reduces
+ *           to add / subtract / skip), §3.2 (fp16 scale per block).
+ *   [sign]  neodrop.ai community round-up, part 2: a Q1_0 model whose weights are
+ *           only +1 or -1, sped up by a dedicated matrix kernel.
+ *   [rht]   feinterview.poetries.top, "27B in 12 GB laptop GPU" article, section
+ *           "12 GB 装下 27B": random Hadamard rotation before low-bit coding
+ *           (QuIP / QuIP# / QTIP lineage).
+ *
+ * Conventions shared by every call
+ *   - A weight matrix is stored one output row per packed row: logical W is K x N
+ *     (K = input features), stored [N][K] with K contiguous; y[n] = sum_k w[n][k] x[k].
+ *   - Pointers are DEVICE pointers unless a comment says otherwise. The caller
+ *     allocates and owns every buffer; the library never allocates, frees or
+ *     synchronises. Calls enqueue on `stream` (a cudaStream_t passed as void*,
+ *     NULL = legacy default stream) and return; results are valid once the
+ *     stream reaches that point.
+ *   - bf16 and fp16 values travel as their raw 16-bit patterns (uint16_t).
+ *   - Every call validates its arguments on the host BEFORE any launch and
+ *     returns a status; on any status other than LBQ_OK nothing was enqueued,
+ *     except LBQ_ERR_CUDA from a failed launch (the launch error is cleared).
+ *     No call aborts, exits or throws across the ABI.
+ *   - Inputs must be finite; NaN/Inf inputs give unspecified (non-faulting) output.
+ *
+ * Packed formats (byte layouts are this library's; the pages fix only the number
+ * system, the block size and the scale rule):
+ *
+ *   LBQ_TERN5 (ternary, [tern] + [block]): blocks of 128 weights, each 28 bytes:
+ *     bytes 0..24  : five trits per byte, little-endian base 3 of d = t + 1:
+ *                    byte j = sum_{i<5} d[5j+i] * 3^i    (weights 5j .. 5j+4)
+ *     byte  25     : weights 125..127 in digits 0..2; digits 3 and 4 are zero
+ *                    trits (d = 1), so the byte is d125 + 3 d126 + 9 d127 + 108
+ *     bytes 26..27 : fp16 scale s16 of the block (little-endian bits)
+ *     Every byte value is <= 242. Rows are padded to a 16-byte multiple
+ *     (code_stride = round_up(28 * K/128, 16)); pad bytes are zero and never read
+ *     for arithmetic. The scale lives inside the block so that every aligned
+ *     32-bit word of a row belongs to exactly one block. `scales` is unused (NULL).
+ *     Quantisation: s16 = fp16_rne(min(mean_k |w_k|, 65504)), mean taken in fp64;
+ *     t = sign(w) if |w| > s16/2 else 0 (equal to clip(round_half_even(w/s16), -1, 1));
+ *     t = 0 everywhere when s16 == 0. Dequantised weight = s16 * t.
+ *
+ *   LBQ_SIGN1 (1-bit, [sign]): codes [N][code_stride], code_stride = K/8 bytes;
+ *     bit i of byte j is weight 8j+i, 1 -> +1, 0 -> -1, bit = (w >= 0).
+ *     scales [N][K/128] fp16, s16 = fp16_rne(min(mean |w|, 65504)) per 128 weights.
+ *     Dequantised weight = s16 * (2 bit - 1).
+ *
+ *   LBQ_Q2RHT (2-bit, 4 levels, rotated input, [rht]): codes [N][K/4] bytes;
+ *     weight 4j+i in bits 2i..2i+1 of byte j; code q in 0..3 means level q - 1.5.
+ *     scales [N][K/32] fp16, s16 = fp16_rne(min(max|w| / 1.5, 65504)) per 32 weights
+ *     (quotient in fp64); q = clip(floor(w/s16) + 2, 0, 3) (nearest level, ties up),
+ *     q = 2 everywhere when s16 == 0. Dequantised weight = s16 * (q - 1.5).
+ *     The weights are expressed in the rotated basis, so the product uses
+ *     x' = H_512 D x / sqrt(512) (see lbq_hadamard) in place of x. K % 512 == 0.
+ *
+ * Shape rules: K % 128 == 0 (LBQ_Q2RHT: K % 512 == 0), K >= 128, N >= 1, M >= 1.
+ * Alignment rules: codes, x/X, W and workspace 16-byte aligned; scales, y/Y and D
+ * 2-byte aligned (D 1-byte). Strides must be at least the packed row size and a
+ * multiple of 16 bytes (codes) / 1 element (scales).
+ */
+#ifndef LBQ_H
+#define LBQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum lbq_status {
+  LBQ_OK = 0,
+  LBQ_ERR_ARG = 1,        /* null pointer or bad enum/flag value            */
+  LBQ_ERR_SHAPE = 2,      /* K, N, M or a stride violates the shape rules  */
+  LBQ_ERR_ALIGN = 3,      /* a pointer violates the alignment rules        */
+  LBQ_ERR_FORMAT = 4,     /* unknown packed format                         */
+  LBQ_ERR_CUDA = 5,       /* a CUDA runtime call or launch failed          */
+  LBQ_ERR_WORKSPACE = 6   /* workspace missing or smaller than required    */
+} lbq_status;
+
+typedef enum lbq_format {
+  LBQ_TERN5 = 1, /* ternary, 5 trits per byte, fp16 scale per 128, in-block     */
+  LBQ_SIGN1 = 2, /* 1-bit sign, fp16 scale per 128, separate scale array       */
+  LBQ_Q2RHT = 3  /* 2-bit 4-level, fp16 scale per 32, input rotated by RHT-512  */
+} lbq_format;
+
+/* A packed weight matrix (descriptor only; the buffers belong to the caller). */
+typedef struct lbq_weights {
+  int32_t fmt;           /* lbq_format                                            */
+  int32_t reserved;      /* must be 0                                             */
+  int64_t K;             /* input features (packed along a row)                   */
+  int64_t N;             /* output features (rows)                                */
+  const void* codes;     /* device, [N][code_stride] bytes                        */
+  const void* scales;    /* device, [N][scale_stride] fp16; NULL for LBQ_TERN5    */
+  int64_t code_stride;   /* bytes between rows of codes                           */
+  int64_t scale_stride;  /* fp16 elements between rows of scales (0 for TERN5)    */
+} lbq_weights;
+
+/* Human-readable name of a status. Never NULL. Host only. */
+const char* lbq_status_string(lbq_status st);
+
+/* Packed sizes for a K x N matrix in format `fmt` (host only, no CUDA call).
+ * Any output pointer may be NULL. code_stride/scale_stride are the minimal
+ * strides; code_bytes = N * code_stride, scale_bytes = N * scale_stride * 2.
+ * Errors: LBQ_ERR_FORMAT, LBQ_ERR_SHAPE. */
+lbq_status lbq_packed_layout(int32_t fmt, int64_t K, int64_t N, int64_t* code_stride,
+                             int64_t* scale_stride, size_t* code_bytes, size_t* scale_bytes);
+
+/* Quantise and pack W (device fp32 [N][K], row-major, 16-byte aligned) into
+ * `codes` ([N][code_stride] bytes) and `scales` ([N][scale_stride] fp16; NULL for
+ * TERN5), using the minimal strides of lbq_packed_layout. Rule per format: see the
+ * header comment ([tern] §5.1 applied per block as in [block] §2.1; [sign]; [rht]).
+ * Deterministic and bit-exact: the same W always gives the same bytes. Offline
+ * step, not tuned for speed. */
+lbq_status lbq_pack(int32_t fmt, const float* W, int64_t K, int64_t N, void* codes,
+                    void* scales, void* stream);
+
+/* Unpack codes to int8 values (t in {-1,0,1} for TERN5, 2b-1 in {-1,1} for SIGN1,
+ * q in {0,1,2,3} for Q2RHT) into out [N][K] (device), and the block scales as fp32
+ * into scales_out [N][K/blk] (device; blk = 128, or 32 for Q2RHT) when non-NULL.
+ * A test hook for the bit-exact code check. */
+lbq_status lbq_unpack(const lbq_weights* w, int8_t* out, float* scales_out, void* stream);
+
+/* Random signs D[k] in {-1,+1}, k < K, for the Hadamard rotation ([rht]):
+ * D[k] = -1 iff bit 63 of the (k+1)-th output of SplitMix64 seeded with `seed`
+ * is set (Steele, Lea & Flood 2014; Vigna's public-domain reference generator).
+ * D is a device int8 array of K elements. */
+lbq_status lbq_rht_signs(uint64_t seed, int64_t K, int8_t* D, void* stream);
+
+/* Block random Hadamard transform of M rows of bf16 activations ([rht]):
+ * out[m][512c+i] = 2^-4.5 * sum_j (-1)^popcount(i&j) * D[512c+j] * x[m][512c+j].
+ * x is [M][K] bf16 (row stride K), out is [M][K] fp32, K % 512 == 0.
+ * Computed with a 9-stage butterfly in shared memory, in fp32. */
+lbq_status lbq_hadamard(const uint16_t* x, const int8_t* D, int64_t M, int64_t K,
+                        float* out, void* stream);
+
+/* Bytes of device workspace lbq_gemv / lbq_gemm need for this matrix and M.
+ * The workspace must be zero-filled before its FIRST use; every call returns it
+ * zero-filled again where that matters, so one zeroing at allocation suffices
+ * for any sequence of completed calls. Calls sharing one workspace must not
+ * overlap in time (use one workspace per stream). Returns 0 on bad arguments. */
+size_t lbq_workspace_bytes(const lbq_weights* w, int64_t M);
+
+/* Batch-1 product y = W_hat x (bf16 x [K] -> bf16 y [N]) with W_hat the dequantised
+ * weights; for LBQ_Q2RHT the input is first rotated, y = W_hat (H D x / sqrt 512),
+ * with D from lbq_rht_signs (NULL for other formats). fp32 accumulation; y is
+ * rounded to bf16 once, at the end. Workspace as lbq_workspace_bytes(w, 1).
+ * Errors: LBQ_ERR_ARG (nulls, D missing for Q2RHT), LBQ_ERR_SHAPE, LBQ_ERR_ALIGN,
+ * LBQ_ERR_FORMAT, LBQ_ERR_WORKSPACE, LBQ_ERR_CUDA. */
+lbq_status lbq_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D, uint16_t* y,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* Batched product Y[m][n] = sum_k W_hat[n][k] X[m][k] for M rows of bf16 X
+ * ([M][K], row stride K) into bf16 Y ([M][N], row stride N). Small M streams the
+ * weights once for all M rows; large M dequantises weight tiles into shared
+ * memory and runs tcgen05 bf16 MMA with fp32 accumulation in tensor memory.
+ * Same formats, D and workspace rules as lbq_gemv (workspace for this M). */
+lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const int8_t* D,
+                    uint16_t* Y, void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LBQ_H */
