@@ -1,0 +1,151 @@
+// api.cu -- the C ABI (include/lbq.h): host-side validation, then one or more launches.
+// Nothing is enqueued unless every argument passes; launch failures map to LBQ_ERR_CUDA.
+#include "lbq_common.cuh"
+
+namespace {
+
+using lbq::Layout;
+
+inline bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+inline lbq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LBQ_OK : LBQ_ERR_CUDA; }
+
+inline bool fmt_known(int32_t fmt) {
+  return fmt == LBQ_TERN5 || fmt == LBQ_SIGN1 || fmt == LBQ_Q2RHT;
+}
+
+// Checks a weight descriptor; fills L on success.
+lbq_status check_weights(const lbq_weights* w, Layout* L) {
+  if (!w) return LBQ_ERR_ARG;
+  if (!fmt_known(w->fmt)) return LBQ_ERR_FORMAT;
+  if (w->reserved != 0) return LBQ_ERR_ARG;
+  if (w->N < 1 || !lbq::layout_of(w->fmt, w->K, L)) return LBQ_ERR_SHAPE;
+  if (!w->codes) return LBQ_ERR_ARG;
+  if (!aligned(w->codes, 16)) return LBQ_ERR_ALIGN;
+  if (w->code_stride < L->code_stride || w->code_stride % 16) return LBQ_ERR_SHAPE;
+  if (w->fmt == LBQ_TERN5) {
+    if (w->scales || w->scale_stride != 0) return LBQ_ERR_ARG;
+  } else {
+    if (!w->scales) return LBQ_ERR_ARG;
+    if (!aligned(w->scales, 2)) return LBQ_ERR_ALIGN;
+    if (w->scale_stride < L->scale_stride) return LBQ_ERR_SHAPE;
+  }
+  return LBQ_OK;
+}
+
+lbq_status check_product(const lbq_weights* w, const void* x, int64_t M, const int8_t* D,
+                         const void* y, void* ws, size_t ws_bytes, Layout* L) {
+  lbq_status st = check_weights(w, L);
+  if (st != LBQ_OK) return st;
+  if (M < 1) return LBQ_ERR_SHAPE;
+  if (!x || !y) return LBQ_ERR_ARG;
+  if (!aligned(x, 16) || !aligned(y, 2)) return LBQ_ERR_ALIGN;
+  if (w->fmt == LBQ_Q2RHT) {
+    if (!D) return LBQ_ERR_ARG;
+    if (!aligned(D, 16)) return LBQ_ERR_ALIGN;
+  }
+  const size_t need = lbq_workspace_bytes(w, M);
+  if (need) {
+    if (!ws || ws_bytes < need) return LBQ_ERR_WORKSPACE;
+    if (!aligned(ws, 16)) return LBQ_ERR_ALIGN;
+  }
+  return LBQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lbq_status_string(lbq_status st) {
+  switch (st) {
+    case LBQ_OK: return "ok";
+    case LBQ_ERR_ARG: return "invalid argument (null pointer or bad value)";
+    case LBQ_ERR_SHAPE: return "invalid shape or stride";
+    case LBQ_ERR_ALIGN: return "misaligned pointer";
+    case LBQ_ERR_FORMAT: return "unknown packed format";
+    case LBQ_ERR_CUDA: return "CUDA error";
+    case LBQ_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+lbq_status lbq_packed_layout(int32_t fmt, int64_t K, int64_t N, int64_t* code_stride,
+                             int64_t* scale_stride, size_t* code_bytes, size_t* scale_bytes) {
+  if (!fmt_known(fmt)) return LBQ_ERR_FORMAT;
+  Layout L;
+  if (N < 1 || !lbq::layout_of(fmt, K, &L)) return LBQ_ERR_SHAPE;
+  if (code_stride) *code_stride = L.code_stride;
+  if (scale_stride) *scale_stride = L.scale_stride;
+  if (code_bytes) *code_bytes = static_cast<size_t>(N) * static_cast<size_t>(L.code_stride);
+  if (scale_bytes) *scale_bytes = static_cast<size_t>(N) * static_cast<size_t>(L.scale_stride) * 2;
+  return LBQ_OK;
+}
+
+lbq_status lbq_pack(int32_t fmt, const float* W, int64_t K, int64_t N, void* codes, void* scales,
+                    void* stream) {
+  if (!fmt_known(fmt)) return LBQ_ERR_FORMAT;
+  Layout L;
+  if (N < 1 || !lbq::layout_of(fmt, K, &L)) return LBQ_ERR_SHAPE;
+  if (!W || !codes) return LBQ_ERR_ARG;
+  if (!aligned(W, 16) || !aligned(codes, 16)) return LBQ_ERR_ALIGN;
+  if (fmt == LBQ_TERN5) {
+    if (scales) return LBQ_ERR_ARG;
+  } else {
+    if (!scales) return LBQ_ERR_ARG;
+    if (!aligned(scales, 2)) return LBQ_ERR_ALIGN;
+  }
+  return from_cuda(lbq_launch_pack(fmt, W, K, N, static_cast<uint8_t*>(codes),
+                                   static_cast<uint16_t*>(scales), L, as_stream(stream)));
+}
+
+lbq_status lbq_unpack(const lbq_weights* w, int8_t* out, float* scales_out, void* stream) {
+  Layout L;
+  lbq_status st = check_weights(w, &L);
+  if (st != LBQ_OK) return st;
+  if (!out) return LBQ_ERR_ARG;
+  if (scales_out && !aligned(scales_out, 4)) return LBQ_ERR_ALIGN;
+  return from_cuda(lbq_launch_unpack(w, L, out, scales_out, as_stream(stream)));
+}
+
+lbq_status lbq_rht_signs(uint64_t seed, int64_t K, int8_t* D, void* stream) {
+  if (!D) return LBQ_ERR_ARG;
+  if (K < 1) return LBQ_ERR_SHAPE;
+  return from_cuda(lbq_launch_rht_signs(seed, K, D, as_stream(stream)));
+}
+
+lbq_status lbq_hadamard(const uint16_t* x, const int8_t* D, int64_t M, int64_t K, float* out,
+                        void* stream) {
+  if (!x || !D || !out) return LBQ_ERR_ARG;
+  if (M < 1 || K < lbq::kRhtBlock || K % lbq::kRhtBlock) return LBQ_ERR_SHAPE;
+  if (!aligned(x, 16) || !aligned(D, 16) || !aligned(out, 16)) return LBQ_ERR_ALIGN;
+  return from_cuda(lbq_launch_hadamard(x, D, M, K, out, as_stream(stream)));
+}
+
+size_t lbq_workspace_bytes(const lbq_weights* w, int64_t M) {
+  Layout L;
+  if (check_weights(w, &L) != LBQ_OK || M < 1) return 0;
+  return M == 1 ? lbq_gemv_workspace(w) : lbq_gemm_workspace(w, M);
+}
+
+lbq_status lbq_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D, uint16_t* y,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  Layout L;
+  lbq_status st = check_product(w, x, 1, D, y, workspace, workspace_bytes, &L);
+  if (st != LBQ_OK) return st;
+  return from_cuda(lbq_launch_gemv(w, x, D, y, workspace, as_stream(stream)));
+}
+
+lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const int8_t* D,
+                    uint16_t* Y, void* workspace, size_t workspace_bytes, void* stream) {
+  Layout L;
+  lbq_status st = check_product(w, X, M, D, Y, workspace, workspace_bytes, &L);
+  if (st != LBQ_OK) return st;
+  if (M == 1) return from_cuda(lbq_launch_gemv(w, X, D, Y, workspace, as_stream(stream)));
+  return from_cuda(lbq_launch_gemm(w, X, M, D, Y, workspace, as_stream(stream)));
+}
+
+}  // extern "C"

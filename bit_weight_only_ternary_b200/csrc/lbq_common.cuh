@@ -1,0 +1,101 @@
+// lbq_common.cuh -- shared device/host helpers of the CUDA library (not of the oracle).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lbq.h"
+
+namespace lbq {
+
+// Layout constants of the packed formats (byte layouts are documented in lbq.h).
+constexpr int kTernBlock = 128;       // weights per ternary block
+constexpr int kTernBlockBytes = 28;   // 26 code bytes + fp16 scale
+constexpr int kTernCodeBytes = 26;
+constexpr int kSignBlock = 128;       // weights per sign scale
+constexpr int kQ2Block = 32;          // weights per 2-bit scale
+constexpr int kRhtBlock = 512;        // Hadamard block size
+// 2^-4.5 = 1/sqrt(512), rounded to fp32.
+constexpr float kRhtNorm = 0.044194173824159216f;
+
+struct Layout {
+  int64_t code_stride;   // bytes per row of codes
+  int64_t scale_stride;  // fp16 scales per row (0: scales in-block)
+  int64_t block;         // weights per scale
+};
+
+// Returns false on an unknown format or a K that violates the shape rules.
+inline bool layout_of(int32_t fmt, int64_t K, Layout* L) {
+  if (K < 128 || K % 128) return false;
+  switch (fmt) {
+    case LBQ_TERN5:
+      L->code_stride = ((K / kTernBlock) * kTernBlockBytes + 15) / 16 * 16;
+      L->scale_stride = 0;
+      L->block = kTernBlock;
+      return true;
+    case LBQ_SIGN1:
+      L->code_stride = K / 8;
+      L->scale_stride = K / kSignBlock;
+      L->block = kSignBlock;
+      return true;
+    case LBQ_Q2RHT:
+      if (K % kRhtBlock) return false;
+      L->code_stride = K / 4;
+      L->scale_stride = K / kQ2Block;
+      L->block = kQ2Block;
+      return true;
+    default:
+      return false;
+  }
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ float f16_bits_to_f32(uint16_t h) {
+  return __half2float(__ushort_as_half(h));
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float v) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+inline int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+}  // namespace lbq
+
+// Launch helpers implemented in the individual .cu files; all return cudaError_t
+// from cudaGetLastError() after the launch.
+cudaError_t lbq_launch_pack(int32_t fmt, const float* W, int64_t K, int64_t N, uint8_t* codes,
+                            uint16_t* scales, const lbq::Layout& L, cudaStream_t s);
+cudaError_t lbq_launch_unpack(const lbq_weights* w, const lbq::Layout& L, int8_t* out,
+                              float* scales_out, cudaStream_t s);
+cudaError_t lbq_launch_rht_signs(uint64_t seed, int64_t K, int8_t* D, cudaStream_t s);
+cudaError_t lbq_launch_hadamard(const uint16_t* x, const int8_t* D, int64_t M, int64_t K,
+                                float* out, cudaStream_t s);
+size_t lbq_gemv_workspace(const lbq_weights* w);
+cudaError_t lbq_launch_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D,
+                            uint16_t* y, void* ws, cudaStream_t s);
+size_t lbq_gemm_workspace(const lbq_weights* w, int64_t M);
+cudaError_t lbq_launch_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const int8_t* D,
+                            uint16_t* Y, void* ws, cudaStream_t s);

@@ -64,9 +64,9 @@
  *     x' = H_512 D x / sqrt(512) (see lbq_hadamard) in place of x. K % 512 == 0.
  *
  * Shape rules: K % 128 == 0 (LBQ_Q2RHT: K % 512 == 0), K >= 128, N >= 1, M >= 1.
- * Alignment rules: codes, x/X, W and workspace 16-byte aligned; scales, y/Y and D
- * 2-byte aligned (D 1-byte). Strides must be at least the packed row size and a
- * multiple of 16 bytes (codes) / 1 element (scales).
+ * Alignment rules: codes, x/X, W, D, out and workspace 16-byte aligned; scales and
+ * y/Y 2-byte aligned. Strides must be at least the packed row size; code strides
+ * a multiple of 16 bytes, scale strides any number of elements.
  */
 #ifndef LBQ_H
 #define LBQ_H

@@ -1,0 +1,229 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Codes must be bit-exact; products must satisfy |y_gpu - y_ref| <= 2^-8 * sum_k |w_hat x|
+per output element, the acceptance bound of the method (y_ref and the bound are the
+oracle's, computed in fp64 from the oracle's own packing of the same seeded W).
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from bit_weight_only_ternary_b200 import synth
+
+pytestmark = pytest.mark.gpu
+TERN5, SIGN1, Q2RHT = 1, 2, 3
+FMTS = (TERN5, SIGN1, Q2RHT)
+TOL = 2.0 ** -8
+NTHREADS = max(1, min(32, os.cpu_count() or 1))
+
+
+@pytest.fixture(scope="module")
+def L():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from bit_weight_only_ternary_b200 import build
+    build.build()
+    from bit_weight_only_ternary_b200 import lbq
+    return lbq
+
+
+def _pack_both(L, orc, fmt, W_cpu):
+    pw = L.lbq_pack(fmt, W_cpu.cuda())
+    codes, scales = orc.pack(fmt, W_cpu.numpy())
+    return pw, codes, scales
+
+
+def _assert_codes_equal(pw, codes, scales):
+    got = pw.codes.cpu().numpy()
+    assert got.shape == codes.shape
+    bad = np.argwhere(got != codes)
+    assert bad.size == 0, f"{len(bad)} code bytes differ, first at {bad[:4].tolist()}"
+    if scales is not None:
+        gs = pw.scales.cpu().numpy().view(np.uint16)
+        assert np.array_equal(gs, scales), "scales differ"
+
+
+def _check_products(y, Y, B, what=""):
+    yg = y.float().cpu().double().numpy().reshape(Y.shape)
+    err = np.abs(yg - Y)
+    lim = TOL * B
+    bad = err > lim
+    if bad.any():
+        i = np.argwhere(bad)[0]
+        pytest.fail(f"{what}: {bad.sum()} of {bad.size} outputs out of bound; first {i.tolist()}: "
+                    f"gpu {yg[tuple(i)]!r} ref {Y[tuple(i)]!r} bound {lim[tuple(i)]!r}")
+    return float((err / np.maximum(lim, 1e-300)).max())
+
+
+def _oracle_D(orc, fmt, K, seed=99):
+    return orc.rht_signs(seed, K) if fmt == Q2RHT else None
+
+
+def _gpu_D(L, fmt, K, seed=99):
+    return L.lbq_rht_signs(seed, K) if fmt == Q2RHT else None
+
+
+# ----------------------------------------------------------------------------- codes
+
+SHAPES = [(256, 512), (37, 1536), (1, 512), (5, 1024)]
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("N,K", SHAPES)
+def test_pack_bit_exact(L, orc, fmt, N, K):
+    W = synth.weights(N, K, 1000 + N + K)
+    pw, codes, scales = _pack_both(L, orc, fmt, W)
+    _assert_codes_equal(pw, codes, scales)
+
+
+@pytest.mark.parametrize("fmt", (TERN5, SIGN1))
+@pytest.mark.parametrize("K", (128, 384, 640))
+def test_pack_ragged_k_and_row_padding(L, orc, fmt, K):
+    W = synth.weights(9, K, 5 + K)
+    pw, codes, scales = _pack_both(L, orc, fmt, W)
+    _assert_codes_equal(pw, codes, scales)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_pack_adversarial_values(L, orc, fmt):
+    K = 512
+    W = synth.weights(8, K, 77)
+    W[0] = 0.0                                   # all-zero row: scale 0
+    W[1, :128] = 0.25                            # ties: |w| = s/2 and w = +-s, -0.0
+    W[1, 0], W[1, 1], W[1, 2], W[1, 3] = 0.125, 0.375, -0.0, -0.25
+    W[1, 4] = -0.125
+    W[2] *= 1e7                                  # scale saturates at 65504
+    W[3] *= 1e-12                                # tiny / subnormal fp16 scales
+    W[4, ::2] = -W[4, 1::2]                      # exact +- pairs
+    W[5, 32:64] = torch.tensor([-1.5, -1.0, -0.5, 0.0, 0.5, 1.0, 1.5, -1.0] * 4)  # 2-bit ties
+    pw, codes, scales = _pack_both(L, orc, fmt, W)
+    _assert_codes_equal(pw, codes, scales)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_unpack_bit_exact(L, orc, fmt):
+    N, K = 33, 1024
+    W = synth.weights(N, K, 4242)
+    pw, codes, scales = _pack_both(L, orc, fmt, W)
+    t, s = L.lbq_unpack(pw)
+    ot, os_ = orc.unpack(fmt, codes, scales, K)
+    assert np.array_equal(t.cpu().numpy(), ot)
+    assert np.array_equal(s.cpu().double().numpy(), os_)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_pack_sampled_rows_of_27b_gate_up(L, orc, fmt):
+    N, K = 2 * synth.FFN, synth.HIDDEN
+    Wd = synth.weights(N, K, 31337, device="cuda")
+    pw = L.lbq_pack(fmt, Wd)
+    rows = torch.tensor([0, 1, 777, 12345, N // 2, N - 2, N - 1])
+    codes, scales = orc.pack(fmt, Wd[rows.cuda()].cpu().numpy())
+    assert np.array_equal(pw.codes[rows.cuda()].cpu().numpy(), codes)
+    if scales is not None:
+        assert np.array_equal(pw.scales[rows.cuda()].cpu().numpy().view(np.uint16), scales)
+
+
+# ----------------------------------------------------------------------------- rotation
+
+@pytest.mark.parametrize("K", (512, 5120, 17408))
+def test_rht_signs_bit_exact(L, orc, K):
+    for seed in (0, 1, 2 ** 63 + 5):
+        assert np.array_equal(L.lbq_rht_signs(seed, K).cpu().numpy(), orc.rht_signs(seed, K))
+
+
+@pytest.mark.parametrize("M,K", [(1, 512), (3, 5120), (2, 17408)])
+def test_hadamard_parity(L, orc, M, K):
+    x = synth.activations(M, K, 55)
+    D = L.lbq_rht_signs(7, K)
+    out = L.lbq_hadamard(x.cuda(), D).cpu().double().numpy()
+    ref = orc.hadamard(x.double().numpy(), orc.rht_signs(7, K))
+    # bound: 2^-8 * sum_{j in block} |x_j| / sqrt(512), per element
+    bsum = np.abs(x.double().numpy()).reshape(M, K // 512, 512).sum(-1) / np.sqrt(512)
+    lim = TOL * np.repeat(bsum, 512, axis=1)
+    assert np.all(np.abs(out - ref) <= lim)
+
+
+# ----------------------------------------------------------------------------- products
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("N,K", SHAPES + [(300, 2048)])
+def test_gemv_parity(L, orc, fmt, N, K):
+    W = synth.weights(N, K, 2000 + N + K)
+    x = synth.activations(1, K, 3000 + K)
+    pw, codes, scales = _pack_both(L, orc, fmt, W)
+    y = L.lbq_gemv(pw, x[0].cuda(), _gpu_D(L, fmt, K))
+    Y, B = orc.gemm(fmt, codes, scales, K, synth.bf16_bits(x), _oracle_D(orc, fmt, K))
+    _check_products(y, Y[0], B[0], f"fmt {fmt} {N}x{K}")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_gemv_one_27b_layer(L, orc, fmt):
+    """Every output of one 27B-shaped layer (QKV, O, gate+up, down), full oracle check."""
+    for mi, (name, K, N) in enumerate(synth.LAYER_SHAPES):
+        Wd = synth.weights(N, K, synth.seed_of(10, 0, mi), device="cuda")
+        pw = L.lbq_pack(fmt, Wd)
+        codes, scales = orc.pack(fmt, Wd.cpu().numpy())
+        del Wd
+        _assert_codes_equal(pw, codes, scales)
+        x = synth.activations(1, K, synth.seed_of(20, 0, mi), device="cuda")
+        y = L.lbq_gemv(pw, x[0], _gpu_D(L, fmt, K))
+        Y, B = orc.gemm(fmt, codes, scales, K, synth.bf16_bits(x), _oracle_D(orc, fmt, K),
+                        nthreads=NTHREADS)
+        _check_products(y, Y[0], B[0], f"fmt {fmt} {name}")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("M", (2, 8, 32, 100))
+def test_gemm_parity(L, orc, fmt, M):
+    N, K = 384, 1536
+    W = synth.weights(N, K, 4000 + M)
+    X = synth.activations(M, K, 5000 + M)
+    pw, codes, scales = _pack_both(L, orc, fmt, W)
+    Yg = L.lbq_gemm(pw, X.cuda(), _gpu_D(L, fmt, K))
+    Y, B = orc.gemm(fmt, codes, scales, K, synth.bf16_bits(X), _oracle_D(orc, fmt, K),
+                    nthreads=NTHREADS)
+    _check_products(Yg, Y, B, f"fmt {fmt} M={M}")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_zero_weights_and_zero_input_give_exact_zero(L, orc, fmt):
+    N, K = 64, 1024
+    W = synth.weights(N, K, 8)
+    W[5:9] = 0.0
+    pw = L.lbq_pack(fmt, W.cuda())
+    x = synth.activations(1, K, 9)[0].cuda()
+    y = L.lbq_gemv(pw, x, _gpu_D(L, fmt, K)).float().cpu()
+    assert torch.all(y[5:9] == 0)
+    y0 = L.lbq_gemv(pw, torch.zeros(K, dtype=torch.bfloat16, device="cuda"), _gpu_D(L, fmt, K))
+    assert torch.all(y0.float() == 0)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_repeated_calls_are_deterministic(L, fmt):
+    N, K = 5120, 5120
+    pw = L.lbq_pack(fmt, synth.weights(N, K, 12, device="cuda"))
+    x = synth.activations(1, K, 13, device="cuda")[0]
+    D = _gpu_D(L, fmt, K)
+    ws = L.workspace_for(pw, 1)
+    a = L.lbq_gemv(pw, x, D, workspace=ws).clone()
+    for _ in range(3):
+        b = L.lbq_gemv(pw, x, D, workspace=ws)
+        assert torch.equal(a, b)
+
+
+def test_errors_enqueue_nothing(L):
+    N, K = 16, 512
+    pw = L.lbq_pack(TERN5, synth.weights(N, K, 3).cuda())
+    x = synth.activations(1, K, 4)[0].cuda()
+    y = torch.full((N,), 7.0, dtype=torch.bfloat16, device="cuda")
+    bad = L.PackedWeights(TERN5, K + 1, N, pw.codes, None)
+    with pytest.raises(L.LbqError) as e:
+        L.lbq_gemv(bad, x, None, y)
+    assert e.value.status == L.LBQ_ERR_SHAPE
+    xb = torch.zeros(K + 8, dtype=torch.bfloat16, device="cuda")[1:K + 1]  # 2-byte offset
+    with pytest.raises(L.LbqError) as e:
+        L.lbq_gemv(pw, xb, None, y)
+    assert e.value.status == L.LBQ_ERR_ALIGN
+    torch.cuda.synchronize()
+    assert torch.all(y.float() == 7.0)
