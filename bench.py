@@ -205,8 +205,9 @@ def ours(args):
         with torch.cuda.graph(graph, stream=stream):
             run_step(L, prods, D, ws, M)
     launches_per_call = 2 if fmt == L.LBQ_Q2RHT else 1  # rotation kernel + product kernel
-    for _ in range(args.warmup):
-        graph.replay()
+    with torch.cuda.stream(stream):  # replays run on the stream the events are recorded on
+        for _ in range(args.warmup):
+            graph.replay()
     torch.cuda.synchronize()
 
     def barrier():
@@ -218,10 +219,11 @@ def ours(args):
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier()
-        t0.record(stream)
-        for _ in range(args.steps):
-            graph.replay()
-        t1.record(stream)
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            t1.record(stream)
         barrier()
     ms = t0.elapsed_time(t1)
     if world > 1:
@@ -277,14 +279,16 @@ def ours(args):
             xin_dev.copy_(xin_host, non_blocking=True)
             run_step(L, e2e_prods, D, ws, M)
             y_host.copy_(y_dev, non_blocking=True)
-    for _ in range(args.warmup):
-        g2.replay()
     e_steps = max(10, args.steps // 4)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            g2.replay()
     barrier()
-    t0.record(stream)
-    for _ in range(e_steps):
-        g2.replay()
-    t1.record(stream)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(e_steps):
+            g2.replay()
+        t1.record(stream)
     barrier()
     ems = t0.elapsed_time(t1)
     if world > 1:
