@@ -21,7 +21,8 @@ LBQ_OK, LBQ_ERR_ARG, LBQ_ERR_SHAPE, LBQ_ERR_ALIGN, LBQ_ERR_FORMAT, LBQ_ERR_CUDA,
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblbq.so")
 EXPORTS = ("lbq_status_string", "lbq_packed_layout", "lbq_pack", "lbq_unpack", "lbq_rht_signs",
-           "lbq_hadamard", "lbq_workspace_bytes", "lbq_gemv", "lbq_gemm")
+           "lbq_hadamard", "lbq_workspace_bytes", "lbq_gemv", "lbq_gemm", "lbq_gemv_noalloc")
+LBQ_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class lbq_weights(ctypes.Structure):
@@ -53,6 +54,7 @@ def _load():
         "lbq_workspace_bytes": (sz, [W, i64]),
         "lbq_gemv": (ctypes.c_int, [W, p, p, p, p, sz, p]),
         "lbq_gemm": (ctypes.c_int, [W, p, i64, p, p, p, sz, p]),
+        "lbq_gemv_noalloc": (ctypes.c_int, [W, p, p, p, p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -193,3 +195,16 @@ def lbq_gemm(pw: PackedWeights, X: torch.Tensor, D=None, Y=None, workspace=None,
     _check(_lib.lbq_gemm(ctypes.byref(d), _ptr(X), M, _ptr(D), _ptr(Y), _ptr(workspace), wsb,
                          _stream(stream)), "lbq_gemm")
     return Y
+
+
+def lbq_gemv_noalloc(pw: PackedWeights, x: torch.Tensor, D=None, y=None,
+                     stream=None) -> torch.Tensor:
+    """lbq_gemv for callers that cannot allocate device memory: the library's own fixed
+    scratch array replaces the workspace (see include/lbq.h). Only `y` is allocated
+    here, and only when the caller passes none."""
+    if y is None:
+        y = torch.empty(pw.N, dtype=torch.bfloat16, device=x.device)
+    d = pw.desc()
+    _check(_lib.lbq_gemv_noalloc(ctypes.byref(d), _ptr(x), _ptr(D), _ptr(y), _stream(stream)),
+           "lbq_gemv_noalloc")
+    return y

@@ -168,6 +168,33 @@ lbq_status lbq_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D, ui
 lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const int8_t* D,
                     uint16_t* Y, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Size of the scratch array that lbq_gemv_noalloc uses (4 MiB). */
+#define LBQ_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* lbq_gemv without a workspace argument, for callers that cannot allocate device
+ * memory: a host that reaches the library only through this C interface and has no
+ * device allocator of its own, or one that must not call cudaMalloc once it is
+ * running (cudaMalloc can synchronise the device, and a framework's memory pool
+ * cannot account for memory taken behind its back). The pages have no counterpart
+ * of this call; it only changes where the scratch memory comes from.
+ *
+ * Same arguments, result and errors as lbq_gemv, minus the workspace. The scratch
+ * is one array of LBQ_NOALLOC_SCRATCH_BYTES compiled into the library: every GPU
+ * that loads the library holds it until the process exits. A call whose product
+ * needs more scratch than that (lbq_workspace_bytes(w, 1)) returns
+ * LBQ_ERR_WORKSPACE and enqueues nothing; use lbq_gemv with your own workspace
+ * then. The call allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ * library routine. It clears the part of the array it uses (an asynchronous
+ * memset on `stream`) before the product.
+ *
+ * The first call on each device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream capture.
+ * All calls on a device share the one array: calls that can overlap on the GPU
+ * (different streams without ordering between them) race on it and give wrong
+ * results. Order them on one stream, or use lbq_gemv with one workspace each. */
+lbq_status lbq_gemv_noalloc(const lbq_weights* w, const uint16_t* x, const int8_t* D,
+                            uint16_t* y, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
