@@ -136,6 +136,7 @@ lbq_status lbq_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D, ui
   Layout L;
   lbq_status st = check_product(w, x, 1, D, y, workspace, workspace_bytes, &L);
   if (st != LBQ_OK) return st;
+  if (lbq_gemv_workspace(w) && w->N > lbq::kMaxSplitRows) return LBQ_ERR_SHAPE;
   return from_cuda(lbq_launch_gemv(w, x, D, y, workspace, as_stream(stream)));
 }
 
@@ -144,7 +145,10 @@ lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const in
   Layout L;
   lbq_status st = check_product(w, X, M, D, Y, workspace, workspace_bytes, &L);
   if (st != LBQ_OK) return st;
-  if (M == 1) return from_cuda(lbq_launch_gemv(w, X, D, Y, workspace, as_stream(stream)));
+  if (M == 1) {
+    if (lbq_gemv_workspace(w) && w->N > lbq::kMaxSplitRows) return LBQ_ERR_SHAPE;
+    return from_cuda(lbq_launch_gemv(w, X, D, Y, workspace, as_stream(stream)));
+  }
   return from_cuda(lbq_launch_gemm(w, X, M, D, Y, workspace, as_stream(stream)));
 }
 

@@ -94,8 +94,9 @@ __global__ void __launch_bounds__(256) gemm_rowwarp(const uint8_t* __restrict__ 
 }  // namespace
 
 size_t lbq_gemm_workspace(const lbq_weights* w, int64_t M) {
-  return w->fmt == LBQ_Q2RHT ? static_cast<size_t>(w->K) * static_cast<size_t>(M) * sizeof(float)
-                             : 0;
+  return w->fmt == LBQ_Q2RHT
+             ? kWsCounterBytes + static_cast<size_t>(w->K) * static_cast<size_t>(M) * sizeof(float)
+             : 0;
 }
 
 cudaError_t lbq_launch_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const int8_t* D,
@@ -116,7 +117,7 @@ cudaError_t lbq_launch_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, 
           codes, w->code_stride, scales, w->scale_stride, w->K, w->N, X, nullptr, M, m_per_cta, Y);
       break;
     default: {
-      float* xr = static_cast<float*>(ws);
+      float* xr = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsCounterBytes);
       cudaError_t e = lbq_launch_hadamard(X, D, M, w->K, xr, s);
       if (e != cudaSuccess) return e;
       gemm_rowwarp<LBQ_Q2RHT><<<grid, 32 * warps, 0, s>>>(

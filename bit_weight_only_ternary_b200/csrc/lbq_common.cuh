@@ -17,6 +17,12 @@ constexpr int kTernCodeBytes = 26;
 constexpr int kSignBlock = 128;       // weights per sign scale
 constexpr int kQ2Block = 32;          // weights per 2-bit scale
 constexpr int kRhtBlock = 512;        // Hadamard block size
+// Workspace layout shared by every product: [0, kWsCounterBytes) holds arrival
+// counters that must be zero when a call starts and are zero again when it ends;
+// the scratch data of a call starts at kWsCounterBytes. Keeping the counters at a
+// fixed place lets one workspace serve matrices of any shape in turn.
+constexpr size_t kWsCounterBytes = 65536;
+constexpr int64_t kMaxSplitRows = static_cast<int64_t>(kWsCounterBytes / 4) * 32;
 // 2^-4.5 = 1/sqrt(512), rounded to fp32.
 constexpr float kRhtNorm = 0.044194173824159216f;
 

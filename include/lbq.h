@@ -63,7 +63,8 @@
  *     The weights are expressed in the rotated basis, so the product uses
  *     x' = H_512 D x / sqrt(512) (see lbq_hadamard) in place of x. K % 512 == 0.
  *
- * Shape rules: K % 128 == 0 (LBQ_Q2RHT: K % 512 == 0), K >= 128, N >= 1, M >= 1.
+ * Shape rules: K % 128 == 0 (LBQ_Q2RHT: K % 512 == 0), K >= 128, N >= 1, M >= 1;
+ * a batch-1 product split over K (K > 512, or > 1024 for LBQ_SIGN1) has N <= 524288.
  * Alignment rules: codes, x/X, W, D, out and workspace 16-byte aligned; scales and
  * y/Y 2-byte aligned. Strides must be at least the packed row size; code strides
  * a multiple of 16 bytes, scale strides any number of elements.
@@ -144,11 +145,12 @@ lbq_status lbq_rht_signs(uint64_t seed, int64_t K, int8_t* D, void* stream);
 lbq_status lbq_hadamard(const uint16_t* x, const int8_t* D, int64_t M, int64_t K,
                         float* out, void* stream);
 
-/* Bytes of device workspace lbq_gemv / lbq_gemm need for this matrix and M.
- * The workspace must be zero-filled before its FIRST use; every call returns it
- * zero-filled again where that matters, so one zeroing at allocation suffices
- * for any sequence of completed calls. Calls sharing one workspace must not
- * overlap in time (use one workspace per stream). Returns 0 on bad arguments. */
+/* Bytes of device workspace lbq_gemv / lbq_gemm need for this matrix and M
+ * (0: none). The first 64 KB of a workspace hold arrival counters: they must be
+ * zero when the workspace is first used, and every completed call leaves them zero
+ * again, so one zero-fill at allocation serves any sequence of calls on matrices
+ * of any shape. The rest is scratch. Calls sharing one workspace must not overlap
+ * in time (use one workspace per stream). Returns 0 on bad arguments. */
 size_t lbq_workspace_bytes(const lbq_weights* w, int64_t M);
 
 /* Batch-1 product y = W_hat x (bf16 x [K] -> bf16 y [N]) with W_hat the dequantised

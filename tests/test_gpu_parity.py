@@ -227,3 +227,28 @@ def test_errors_enqueue_nothing(L):
     assert e.value.status == L.LBQ_ERR_ALIGN
     torch.cuda.synchronize()
     assert torch.all(y.float() == 7.0)
+
+
+def test_one_workspace_serves_products_of_any_shape(L, orc):
+    """One zero-filled workspace used in turn by products of different shapes, formats and M
+    (the counters at its start must survive every other product's scratch data)."""
+    cases = [(TERN5, 4352, 5120, 1), (TERN5, 640, 17408, 1), (SIGN1, 3000, 5120, 1),
+             (Q2RHT, 700, 5120, 1), (TERN5, 2000, 1024, 1), (Q2RHT, 96, 1024, 4),
+             (SIGN1, 5000, 2048, 1)]
+    built = []
+    for i, (fmt, N, K, M) in enumerate(cases):
+        W = synth.weights(N, K, 9100 + i)
+        X = synth.activations(M, K, 9200 + i)
+        pw, codes, scales = _pack_both(L, orc, fmt, W)
+        Y, B = orc.gemm(fmt, codes, scales, K, synth.bf16_bits(X), _oracle_D(orc, fmt, K),
+                        nthreads=NTHREADS)
+        built.append((pw, X.cuda(), _gpu_D(L, fmt, K), Y, B, M))
+    need = max(L.lbq_workspace_bytes(pw, M) for pw, _, _, _, _, M in built)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for order in (built, built[::-1], built):
+        for pw, X, D, Y, B, M in order:
+            out = L.lbq_gemv(pw, X[0], D, workspace=ws) if M == 1 else \
+                L.lbq_gemm(pw, X, D, workspace=ws)
+            _check_products(out, Y if M > 1 else Y[0], B if M > 1 else B[0], f"shared ws {pw.N}x{pw.K}")
+    torch.cuda.synchronize()
+    assert not ws[:65536].any(), "counters not left at zero"
