@@ -31,8 +31,8 @@ lbq_status check_weights(const lbq_weights* w, Layout* L) {
     if (w->scales || w->scale_stride != 0) return LBQ_ERR_ARG;
   } else {
     if (!w->scales) return LBQ_ERR_ARG;
-    if (!aligned(w->scales, 2)) return LBQ_ERR_ALIGN;
-    if (w->scale_stride < L->scale_stride) return LBQ_ERR_SHAPE;
+    if (!aligned(w->scales, 16)) return LBQ_ERR_ALIGN;
+    if (w->scale_stride < L->scale_stride || w->scale_stride % 8) return LBQ_ERR_SHAPE;
   }
   return LBQ_OK;
 }
@@ -96,7 +96,7 @@ lbq_status lbq_pack(int32_t fmt, const float* W, int64_t K, int64_t N, void* cod
     if (scales) return LBQ_ERR_ARG;
   } else {
     if (!scales) return LBQ_ERR_ARG;
-    if (!aligned(scales, 2)) return LBQ_ERR_ALIGN;
+    if (!aligned(scales, 16)) return LBQ_ERR_ALIGN;
   }
   return from_cuda(lbq_launch_pack(fmt, W, K, N, static_cast<uint8_t*>(codes),
                                    static_cast<uint16_t*>(scales), L, as_stream(stream)));
@@ -123,6 +123,17 @@ lbq_status lbq_hadamard(const uint16_t* x, const int8_t* D, int64_t M, int64_t K
   if (M < 1 || K < lbq::kRhtBlock || K % lbq::kRhtBlock) return LBQ_ERR_SHAPE;
   if (!aligned(x, 16) || !aligned(D, 16) || !aligned(out, 16)) return LBQ_ERR_ALIGN;
   return from_cuda(lbq_launch_hadamard(x, D, M, K, out, as_stream(stream)));
+}
+
+lbq_status lbq_device_fault(uint32_t* code) {
+  if (!code) return LBQ_ERR_ARG;
+  unsigned* word = lbq_fault_word();
+  if (!word) return LBQ_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpy(&v, word, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return LBQ_ERR_CUDA;
+  if (v && cudaMemset(word, 0, sizeof(v)) != cudaSuccess) return LBQ_ERR_CUDA;
+  *code = v;
+  return LBQ_OK;
 }
 
 size_t lbq_workspace_bytes(const lbq_weights* w, int64_t M) {

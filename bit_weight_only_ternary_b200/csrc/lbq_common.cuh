@@ -43,7 +43,7 @@ inline bool layout_of(int32_t fmt, int64_t K, Layout* L) {
       return true;
     case LBQ_SIGN1:
       L->code_stride = K / 8;
-      L->scale_stride = K / kSignBlock;
+      L->scale_stride = (K / kSignBlock + 7) / 8 * 8;  // 16-byte rows of scales
       L->block = kSignBlock;
       return true;
     case LBQ_Q2RHT:
@@ -100,6 +100,8 @@ cudaError_t lbq_launch_rht_signs(uint64_t seed, int64_t K, int8_t* D, cudaStream
 cudaError_t lbq_launch_hadamard(const uint16_t* x, const int8_t* D, int64_t M, int64_t K,
                                 float* out, cudaStream_t s);
 size_t lbq_gemv_workspace(const lbq_weights* w);
+// Device address of the word bounded device waits report to (current device), or NULL.
+unsigned* lbq_fault_word();
 cudaError_t lbq_launch_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D,
                             uint16_t* y, void* ws, cudaStream_t s);
 size_t lbq_gemm_workspace(const lbq_weights* w, int64_t M);

@@ -89,6 +89,8 @@ __global__ void pack_sign_kernel(const float* __restrict__ W, int64_t K, int64_t
   const int64_t n = gid / nb, b = gid % nb;
   const float* w = W + n * K + b * kSignBlock;
   scales[n * sstride + b] = scale_to_f16_bits(abs_sum<kSignBlock>(w) / 128.0);
+  if (b == nb - 1)  // zero the scale-row padding
+    for (int64_t p = nb; p < sstride; ++p) scales[n * sstride + p] = 0;
   uint32_t* o32 = reinterpret_cast<uint32_t*>(codes + n * cstride + b * 16);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {

@@ -17,11 +17,11 @@ LBQ_TERN5, LBQ_SIGN1, LBQ_Q2RHT = 1, 2, 3
 FORMATS = {"tern": LBQ_TERN5, "sign": LBQ_SIGN1, "q2": LBQ_Q2RHT}
 
 LBQ_OK, LBQ_ERR_ARG, LBQ_ERR_SHAPE, LBQ_ERR_ALIGN, LBQ_ERR_FORMAT, LBQ_ERR_CUDA, \
-    LBQ_ERR_WORKSPACE = range(7)
+    LBQ_ERR_WORKSPACE, LBQ_ERR_DEVICE_WAIT = range(8)
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblbq.so")
 EXPORTS = ("lbq_status_string", "lbq_packed_layout", "lbq_pack", "lbq_unpack", "lbq_rht_signs",
-           "lbq_hadamard", "lbq_workspace_bytes", "lbq_gemv", "lbq_gemm", "lbq_gemv_noalloc")
+           "lbq_hadamard", "lbq_workspace_bytes", "lbq_gemv", "lbq_gemm", "lbq_gemv_noalloc", "lbq_device_fault")
 LBQ_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -55,6 +55,7 @@ def _load():
         "lbq_gemv": (ctypes.c_int, [W, p, p, p, p, sz, p]),
         "lbq_gemm": (ctypes.c_int, [W, p, i64, p, p, p, sz, p]),
         "lbq_gemv_noalloc": (ctypes.c_int, [W, p, p, p, p]),
+        "lbq_device_fault": (ctypes.c_int, [p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -123,6 +124,7 @@ def lbq_pack(fmt: int, W: torch.Tensor, stream=None) -> PackedWeights:
     cs, ss, cb, sb = lbq_packed_layout(fmt, K, N)
     codes = torch.empty((N, cs), dtype=torch.uint8, device=W.device)
     scales = torch.empty((N, ss), dtype=torch.int16, device=W.device) if ss else None
+    # (torch's allocations are 256-byte aligned, as the scales' TMA rows require)
     _check(_lib.lbq_pack(fmt, _ptr(W), K, N, _ptr(codes), _ptr(scales), _stream(stream)),
            "lbq_pack")
     return PackedWeights(fmt, K, N, codes, scales)
@@ -152,6 +154,13 @@ def lbq_hadamard(x: torch.Tensor, D: torch.Tensor, out=None, stream=None) -> tor
         out = torch.empty((M, K), dtype=torch.float32, device=x.device)
     _check(_lib.lbq_hadamard(_ptr(x2), _ptr(D), M, K, _ptr(out), _stream(stream)), "lbq_hadamard")
     return out.view(x.shape)
+
+
+def lbq_device_fault() -> int:
+    """Code of a bounded in-kernel wait that gave up since the last query (0: none)."""
+    code = ctypes.c_uint32()
+    _check(_lib.lbq_device_fault(ctypes.byref(code)), "lbq_device_fault")
+    return code.value
 
 
 def lbq_workspace_bytes(pw: PackedWeights, M: int = 1) -> int:

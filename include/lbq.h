@@ -52,7 +52,9 @@
  *
  *   LBQ_SIGN1 (1-bit, [sign]): codes [N][code_stride], code_stride = K/8 bytes;
  *     bit i of byte j is weight 8j+i, 1 -> +1, 0 -> -1, bit = (w >= 0).
- *     scales [N][K/128] fp16, s16 = fp16_rne(min(mean |w|, 65504)) per 128 weights.
+ *     scales [N][scale_stride] fp16 with scale_stride = round_up(K/128, 8) (rows of
+ *     scales padded with zeros to 16 bytes), s16 = fp16_rne(min(mean |w|, 65504))
+ *     per 128 weights.
  *     Dequantised weight = s16 * (2 bit - 1).
  *
  *   LBQ_Q2RHT (2-bit, 4 levels, rotated input, [rht]): codes [N][K/4] bytes;
@@ -65,9 +67,10 @@
  *
  * Shape rules: K % 128 == 0 (LBQ_Q2RHT: K % 512 == 0), K >= 128, N >= 1, M >= 1;
  * a batch-1 product split over K (K > 512, or > 1024 for LBQ_SIGN1) has N <= 524288.
- * Alignment rules: codes, x/X, W, D, out and workspace 16-byte aligned; scales and
- * y/Y 2-byte aligned. Strides must be at least the packed row size; code strides
- * a multiple of 16 bytes, scale strides any number of elements.
+ * Alignment rules: codes, scales, x/X, W, D, out and workspace 16-byte aligned;
+ * y/Y 2-byte aligned. Strides must be at least the packed row size; code strides a
+ * multiple of 16 bytes, scale strides a multiple of 8 elements (16 bytes): the
+ * kernels stream both with TMA.
  */
 #ifndef LBQ_H
 #define LBQ_H
@@ -86,7 +89,8 @@ typedef enum lbq_status {
   LBQ_ERR_ALIGN = 3,      /* a pointer violates the alignment rules        */
   LBQ_ERR_FORMAT = 4,     /* unknown packed format                         */
   LBQ_ERR_CUDA = 5,       /* a CUDA runtime call or launch failed          */
-  LBQ_ERR_WORKSPACE = 6   /* workspace missing or smaller than required    */
+  LBQ_ERR_WORKSPACE = 6,  /* workspace missing or smaller than required    */
+  LBQ_ERR_DEVICE_WAIT = 7 /* a bounded wait inside a kernel gave up        */
 } lbq_status;
 
 typedef enum lbq_format {
@@ -172,6 +176,15 @@ lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const in
 
 /* Size of the scratch array that lbq_gemv_noalloc uses (4 MiB). */
 #define LBQ_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* Reports whether a bounded wait inside one of the library's kernels gave up on the
+ * current device since the last query, and clears that record. Every wait in the
+ * kernels (on an mbarrier, for a TMA copy or a slot) is bounded by about 2 s; a
+ * wait that runs out records a non-zero *code (1: producer, 2: consumer, 3: shared
+ * memory layout) and the kernel returns early with incomplete outputs instead of
+ * hanging. A non-zero code means a library fault. Synchronises the device.
+ * Errors: LBQ_ERR_ARG (code NULL), LBQ_ERR_CUDA. */
+lbq_status lbq_device_fault(uint32_t* code);
 
 /* lbq_gemv without a workspace argument, for callers that cannot allocate device
  * memory: a host that reaches the library only through this C interface and has no

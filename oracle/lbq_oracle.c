@@ -75,7 +75,8 @@ double orc_bf16_to_f64(uint16_t b) {
 
 /* Format 1 (ternary): 128-weight blocks of 28 bytes = 26 code bytes + fp16 scale,
  *   rows padded to 16 bytes. Format 2 (sign): K/8 code bytes per row, one fp16
- *   scale per 128. Format 3 (2-bit): K/4 code bytes per row, one fp16 scale per 32. */
+ *   scale per 128, scale rows padded with zeros to a multiple of 8 entries.
+ *   Format 3 (2-bit): K/4 code bytes per row, one fp16 scale per 32. */
 int orc_layout(int fmt, int64_t K, int64_t* code_stride, int64_t* scale_stride,
                int64_t* block) {
   int64_t cs, ss, blk;
@@ -87,7 +88,7 @@ int orc_layout(int fmt, int64_t K, int64_t* code_stride, int64_t* scale_stride,
     blk = 128;
   } else if (fmt == 2) {
     cs = K / 8;
-    ss = K / 128;
+    ss = (K / 128 + 7) / 8 * 8; /* scale rows padded to 8 entries (16 bytes), pad = 0 */
     blk = 128;
   } else if (fmt == 3) {
     if (K % 512) return -1;
@@ -156,6 +157,7 @@ int orc_pack(int fmt, const float* W, int64_t K, int64_t N, uint8_t* codes,
   if (!W || !codes || N < 1 || orc_layout(fmt, K, &cs, &ss, &blk)) return -1;
   if (fmt != 1 && !scales) return -1;
   memset(codes, 0, (size_t)(N * cs));
+  if (scales) memset(scales, 0, sizeof(uint16_t) * (size_t)(N * ss));
   for (int64_t n = 0; n < N; ++n) {
     const float* wr = W + n * K;
     uint8_t* cr = codes + n * cs;

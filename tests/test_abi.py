@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for st in range(7):
+    for st in range(8):
         assert L.lbq_status_string(st)
     assert L.lbq_status_string(99) == "unknown status"
 
@@ -91,11 +91,11 @@ def test_validation_rejects_before_launch(L):
     assert lib.lbq_gemv(ctypes.byref(ok), x, None, ctypes.c_void_p(0x30001), None, 0,
                         None) == L.LBQ_ERR_ALIGN
     assert lib.lbq_gemm(ctypes.byref(ok), x, 0, None, y, None, 0, None) == L.LBQ_ERR_SHAPE
-    sign = _desc(L, fmt=2, scales=None, ss=4)
+    sign = _desc(L, fmt=2, scales=None, ss=8)
     assert lib.lbq_gemv(ctypes.byref(sign), x, None, y, None, 0, None) == L.LBQ_ERR_ARG
     sign = _desc(L, fmt=2, scales=0x60000, ss=3)
     assert lib.lbq_gemv(ctypes.byref(sign), x, None, y, None, 0, None) == L.LBQ_ERR_SHAPE
-    sign = _desc(L, fmt=2, scales=0x60001, ss=4)
+    sign = _desc(L, fmt=2, scales=0x60008, ss=8)
     assert lib.lbq_gemv(ctypes.byref(sign), x, None, y, None, 0, None) == L.LBQ_ERR_ALIGN
     q2 = _desc(L, fmt=3, scales=0x60000, ss=16)
     assert lib.lbq_gemv(ctypes.byref(q2), x, None, y, None, 0, None) == L.LBQ_ERR_ARG  # no D
@@ -121,3 +121,4 @@ def test_validation_rejects_before_launch(L):
     assert lib.lbq_hadamard(x, D, 1, 512, ctypes.c_void_p(0x30004), None) == L.LBQ_ERR_ALIGN
     assert lib.lbq_rht_signs(1, 0, D, None) == L.LBQ_ERR_SHAPE
     assert lib.lbq_rht_signs(1, 5, None, None) == L.LBQ_ERR_ARG
+    assert lib.lbq_device_fault(None) == L.LBQ_ERR_ARG

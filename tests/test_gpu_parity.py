@@ -252,3 +252,9 @@ def test_one_workspace_serves_products_of_any_shape(L, orc):
             _check_products(out, Y if M > 1 else Y[0], B if M > 1 else B[0], f"shared ws {pw.N}x{pw.K}")
     torch.cuda.synchronize()
     assert not ws[:65536].any(), "counters not left at zero"
+
+
+def test_no_bounded_device_wait_gave_up(L):
+    """After every product above, no in-kernel wait ran out (the fault record is clear)."""
+    torch.cuda.synchronize()
+    assert L.lbq_device_fault() == 0
