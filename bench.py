@@ -44,7 +44,10 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 # dram bytes per launch of the dominant kernel from one ncu capture (one 27B layer, the
 # four products, averaged per launch), keyed by the hash of the kernel source it was
 # taken on; reported as null once that source changes.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/gemv_tern_1layer_full.md: 72.42 MB read + 1.3 KB written over the 4 launches
+    ("tern", "ad149e3ac4779581"): 18.105e6,
+}
 
 
 def parse():
@@ -75,12 +78,18 @@ def peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def kernel_source_hash():
+GEMV_SOURCES = ("gemv.cu", "rht.cuh", "sm100_async.cuh", "lbq_common.cuh")
+GEMM_SOURCES = ("gemm.cu", "sm100_async.cuh", "lbq_common.cuh")
+
+
+def kernel_source_hash(files=GEMV_SOURCES):
+    """Hash of the kernel sources a workload runs (keys the recorded ncu traffic)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_weight_only_ternary_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in files:
+        p = os.path.join(csrc, f)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -204,7 +213,9 @@ def ours(args):
         torch.cuda.synchronize()
         with torch.cuda.graph(graph, stream=stream):
             run_step(L, prods, D, ws, M)
-    launches_per_call = 2 if fmt == L.LBQ_Q2RHT else 1  # rotation kernel + product kernel
+    # kernels per product: the GEMV, plus the split-K sum when K spans several slices
+    per_slice = 1024 if fmt == L.LBQ_SIGN1 else 512
+    launches = sum(1 + (p["K"] > per_slice) for p in prods) if M == 1 else len(prods)
     with torch.cuda.stream(stream):  # replays run on the stream the events are recorded on
         for _ in range(args.warmup):
             graph.replay()
@@ -253,7 +264,7 @@ def ours(args):
             "kernel": "lbq_gemv (%s)" % args.workload,
             "algorithmic_bytes_per_launch": algo_bytes / len(prods),
             "avg_launch_us": round(1e3 * kern_ms / len(prods), 3)}
-    key = kernel_source_hash()
+    key = kernel_source_hash(GEMV_SOURCES if M == 1 else GEMM_SOURCES)
     tr = NCU_TRAFFIC.get((args.workload, key))
     roof["traffic"] = tr
     if M >= 512:
@@ -331,7 +342,7 @@ def ours(args):
                    "l2": "inputs larger than L2 (no flush): %.2f GB of weights per step"
                          % (weight_bytes / 1e9),
                    "parallelism": f"replicas x{world}", "graph": "one CUDA graph per step"},
-        "roofline": roof, "e2e": e2e, "gpu_launches": args.steps * len(prods) * launches_per_call,
+        "roofline": roof, "e2e": e2e, "gpu_launches": args.steps * launches,
         "clocks": clocks, "parity": parity, "cpu_baseline": cpu, "kernel_source": key,
     }
     if M > 1:

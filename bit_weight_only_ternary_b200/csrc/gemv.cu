@@ -22,12 +22,15 @@
 //    works on row g ^ l of the unit (rows visited in Gray-code order, so the row
 //    address moves by one signed power of two per step); every read stays
 //    conflict-free and a select-free butterfly then leaves row l's sum in lane l.
-//  * Split-K. Slices are spread over CTAs; each unit's 32 sums go to the workspace
-//    and the last warp to finish a 32-row chunk (a counter per chunk in the fixed
-//    counter region) adds the slices in a fixed order and writes bf16 y: results
-//    are deterministic, and that warp resets the counter.
-//  * Persistent grid, one 544-thread CTA per SM with an equal share of the
-//    (slice, chunk) units in slice-major order. Programmatic dependent launch:
+//  * Split-K. Slices are spread over CTAs; each unit's 32 sums go to the workspace,
+//    and a small second kernel (launched with programmatic dependent launch, so it
+//    starts while the first is finishing) adds each row's slice sums in slice order
+//    and writes bf16 y: results are deterministic. (Folding that sum into the main
+//    kernel, with the last of a row group's CTAs doing it, measured slightly slower.)
+//    A matrix of one slice writes y directly.
+//  * Grid of floor(SMs / slices) CTAs per slice, one CTA per SM, each with an equal
+//    share of its slice's 32-row chunks, so that no CTA builds a second table.
+//    Programmatic dependent launch:
 //    the producer streams weights before the previous kernel in the stream has
 //    finished; consumers wait for it before touching x, y or the workspace.
 #include <cudaTypedefs.h>
@@ -39,21 +42,29 @@ namespace {
 
 using namespace lbq;
 
-constexpr int kConsumers = 16;                  // consumer warps
-constexpr int kThreads = 32 * (kConsumers + 1); // + one producer warp
+constexpr int kMaxConsumers = 16;               // consumer warps (per format, see Traits)
+constexpr int kMaxThreads = 32 * (kMaxConsumers + 1);  // + one producer warp
 constexpr int kRows = 32;                       // rows per unit
-constexpr int kStages = 16;                     // units in flight per CTA
+constexpr int kMaxStages = 32;
 constexpr uint32_t kPage = 65536;               // table page: 256 values x 256 bytes
-constexpr uint32_t kStageCodes = 4096;          // 32 rows x 128 bytes (ternary uses 112)
-constexpr uint32_t kStageBytes = kStageCodes + 1024;  // + 32 rows x 32 bytes of scales
-constexpr uint32_t kTailBytes = 4096 + 2 * kStages * 8;  // x slice + mbarriers
+constexpr uint32_t kTailBytes = 4096 + 2 * kMaxStages * 8;  // x slice + mbarriers
 // Shared memory layout. The table must start on a 64 KB boundary of the shared
 // window (its page addressing keeps the base in the upper half of the PRMT
 // operand), and the dynamic allocation does not start on one (the first 1 KB of
 // the window is reserved). So the whole opt-in maximum is requested: the table
 // sits at the first 64 KB boundary, the stages fill the space below it and
-// continue above it, followed by the x slice and the mbarriers.
-constexpr size_t kSmem = 232448;
+// continue above it, followed by the x slice and the mbarriers. There are more
+// stages than consumer warps, so each warp's next unit streams in while it works
+// on the current one. The request is sized for a window starting at 0 or 1 KB, and
+// leaves room on the SM for a CTA of the small split-K sum kernel.
+constexpr uint32_t smem_bytes(uint32_t stage, uint32_t stages) {
+  // window starting at 1 KB: stages below the table, the rest above it
+  const uint32_t below = (kPage - 1024) / stage < stages ? (kPage - 1024) / stage : stages;
+  const uint32_t at_1k = (kPage - 1024) + 2 * kPage + (stages - below) * stage + kTailBytes;
+  // window starting at 0: everything above the table
+  const uint32_t at_0 = 2 * kPage + stages * stage + kTailBytes;
+  return at_1k > at_0 ? at_1k : at_0;
+}
 constexpr unsigned kFaultProducer = 1, kFaultConsumer = 2, kFaultLayout = 3;
 
 template <int FMT>
@@ -63,18 +74,30 @@ struct Traits<LBQ_TERN5> {
   static constexpr int kWeights = 512, kBlocks = 4, kPitch = 112;
   static constexpr int kHi = 9;                 // value = lo + 27 * hi
   static constexpr int kScaleBox = 0;           // scales live in the blocks
+  static constexpr uint32_t kStageCodes = 3584, kStageBytes = 3584;  // 32 x 112 bytes
+  static constexpr int kStages = 26;
+  static constexpr int kConsumers = 16;
+  static constexpr uint32_t kSmem = smem_bytes(kStageBytes, kStages);
 };
 template <>
 struct Traits<LBQ_SIGN1> {
   static constexpr int kWeights = 1024, kBlocks = 8, kPitch = 128;
   static constexpr int kHi = 16;                // value = lo + 16 * hi
   static constexpr int kScaleBox = 8;           // fp16 scales per row per slice
+  static constexpr uint32_t kStageCodes = 4096, kStageBytes = 4096 + 512;
+  static constexpr int kStages = 20;
+  static constexpr int kConsumers = 14;
+  static constexpr uint32_t kSmem = smem_bytes(kStageBytes, kStages);
 };
 template <>
 struct Traits<LBQ_Q2RHT> {
   static constexpr int kWeights = 512, kBlocks = 16, kPitch = 128;
   static constexpr int kHi = 16;
   static constexpr int kScaleBox = 16;
+  static constexpr uint32_t kStageCodes = 4096, kStageBytes = 4096 + 1024;
+  static constexpr int kStages = 18;
+  static constexpr int kConsumers = 12;
+  static constexpr uint32_t kSmem = smem_bytes(kStageBytes, kStages);
 };
 
 template <uint32_t kImm>
@@ -97,15 +120,20 @@ __device__ __forceinline__ void sts_f2(uint32_t addr, float2 v) {
   asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(v.x), "f"(v.y) : "memory");
 }
 
-// The four table entries addressed by the bytes of `word`, as (e0 + e1, e2 + e3).
-// Slot i lives on page i/2 at column offset (i%2)*128; `lanereg` = table base | lane*4.
-__device__ __forceinline__ void lookup4(uint32_t word, uint32_t lanereg, float& a, float& b) {
-  const float e0 = lds_imm<0>(__byte_perm(word, lanereg, 0x7604));
-  const float e1 = lds_imm<128>(__byte_perm(word, lanereg, 0x7614));
-  const float e2 = lds_imm<kPage>(__byte_perm(word, lanereg, 0x7624));
-  const float e3 = lds_imm<kPage + 128>(__byte_perm(word, lanereg, 0x7634));
-  a = e0 + e1;
-  b = e2 + e3;
+// Sum of the four table entries addressed by the bytes of w0 (.x) and of w1 (.y),
+// two rows at a time so the adds run packed. Slot i lives on page i/2 at column
+// offset (i%2)*128; `lanereg` = table base | lane*4.
+template <uint32_t kImm, uint32_t kSel>
+__device__ __forceinline__ float2 entry2(uint32_t w0, uint32_t w1, uint32_t lanereg) {
+  return make_float2(lds_imm<kImm>(__byte_perm(w0, lanereg, kSel)),
+                     lds_imm<kImm>(__byte_perm(w1, lanereg, kSel)));
+}
+__device__ __forceinline__ float2 lookup4x2(uint32_t w0, uint32_t w1, uint32_t lanereg) {
+  const float2 e0 = entry2<0, 0x7604>(w0, w1, lanereg);
+  const float2 e1 = entry2<128, 0x7614>(w0, w1, lanereg);
+  const float2 e2 = entry2<kPage, 0x7624>(w0, w1, lanereg);
+  const float2 e3 = entry2<kPage + 128, 0x7634>(w0, w1, lanereg);
+  return __fadd2_rn(__fadd2_rn(e0, e1), __fadd2_rn(e2, e3));
 }
 
 // Weight index (within the slice) of digit e of the byte in table column (slot, w),
@@ -147,70 +175,112 @@ struct Args {
   const int8_t* D;
   uint16_t* y;
   float* part;    // [KS][N] slice sums (KS > 1)
-  uint32_t* cnt;  // [NC] per-chunk arrival counters (KS > 1)
   int KS;         // number of slices
+  int G;          // CTAs per slice
   int nblk;       // scale blocks per row
   unsigned* fault;  // set when a bounded wait gives up
 };
 
 // Builds the x slice and the lookup tables for slice j (consumer threads only).
+// Thread t owns table column pair t % 64 (two adjacent lanes of one byte slot) and
+// the values v = lo + R * hi for hi = t / 64, t / 64 + T/64, ...; everything that
+// does not depend on hi is computed once.
 template <int FMT>
-__device__ __forceinline__ void build_slice(const Args<FMT>& a, int64_t j, uint32_t tbase,
+__device__ __forceinline__ void build_slice(const Args<FMT>& a, int32_t j, uint32_t tbase,
                                             float* xs, int ctid) {
   using T = Traits<FMT>;
-  const int64_t blk0 = j * T::kBlocks;
-  const int nb_here = static_cast<int>(a.nblk - blk0 < T::kBlocks ? a.nblk - blk0 : T::kBlocks);
+  constexpr int kCT = 32 * T::kConsumers;
+  const int blk0 = j * T::kBlocks;
+  const int nb_here = a.nblk - blk0 < T::kBlocks ? a.nblk - blk0 : T::kBlocks;
   const int nw = FMT == LBQ_TERN5 ? 7 * nb_here : (FMT == LBQ_SIGN1 ? 4 * nb_here : 2 * nb_here);
   const int nx = FMT == LBQ_Q2RHT ? nb_here * kQ2Block : nb_here * kTernBlock;
-  const int64_t k0 = j * T::kWeights;
+  const int64_t k0 = static_cast<int64_t>(j) * T::kWeights;
   const int lane = ctid & 31;
 
   if (FMT == LBQ_Q2RHT) {
     if (ctid < 32) {
       float v[16];
       rht512_warp_load(a.x + k0, a.D + k0, v);
+      float4* d = reinterpret_cast<float4*>(xs + 16 * lane);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) xs[16 * lane + i] = v[i];
+      for (int q = 0; q < 4; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
   } else {
-    for (int i = ctid; i < T::kWeights; i += 32 * kConsumers)
-      xs[i] = i < nx ? bf16_bits_to_f32(a.x[k0 + i]) : 0.0f;
-  }
-  named_bar_sync(1, 32 * kConsumers);
-
-  for (int task = ctid; task < 64 * T::kHi; task += 32 * kConsumers) {
-    const int cp = task & 63, hi = task >> 6;
-    const int slot = cp >> 4, w0 = 2 * (cp & 15);
-    constexpr int kDigits = FMT == LBQ_TERN5 ? 5 : (FMT == LBQ_SIGN1 ? 8 : 4);
-    float2 xv[kDigits];
+    // one 16-byte load of 8 activations per thread (x is 16-byte aligned, slices too)
+    for (int i = ctid; i < T::kWeights / 8; i += kCT) {
+      float f[8];
+      if (8 * i < nx) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x + k0) + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int e = 0; e < kDigits; ++e) {
-      const int ka = digit_weight<FMT>(slot, w0, e, nw);
-      const int kb = digit_weight<FMT>(slot, w0 + 1, e, nw);
-      xv[e] = make_float2(ka >= 0 ? xs[ka] : 0.0f, kb >= 0 ? xs[kb] : 0.0f);
+        for (int q = 0; q < 4; ++q) {
+          f[2 * q] = __uint_as_float(w[q] << 16);
+          f[2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) f[q] = 0.0f;
+      }
+      float4* d = reinterpret_cast<float4*>(xs + 8 * i);
+      d[0] = make_float4(f[0], f[1], f[2], f[3]);
+      d[1] = make_float4(f[4], f[5], f[6], f[7]);
     }
-    const uint32_t col = tbase + (slot >> 1) * kPage + (slot & 1) * 128 + w0 * 4;
-    if (FMT == LBQ_TERN5) {
-      // v = d0 + 3 d1 + 9 d2 + 27 (d3 + 3 d4); entry = sum_e (d_e - 1) x_e
+  }
+  named_bar_sync(1, kCT);
+
+  const int cp = ctid & 63;
+  const int slot = cp >> 4, w0 = 2 * (cp & 15);
+  constexpr int kDigits = FMT == LBQ_TERN5 ? 5 : (FMT == LBQ_SIGN1 ? 8 : 4);
+  float2 xv[kDigits];
+#pragma unroll
+  for (int e = 0; e < kDigits; ++e) {
+    const int ka = digit_weight<FMT>(slot, w0, e, nw);
+    const int kb = digit_weight<FMT>(slot, w0 + 1, e, nw);
+    xv[e] = make_float2(ka >= 0 ? xs[ka] : 0.0f, kb >= 0 ? xs[kb] : 0.0f);
+  }
+  const uint32_t col = tbase + (slot >> 1) * kPage + (slot & 1) * 128 + w0 * 4;
+  if (FMT == LBQ_TERN5) {
+    // v = d0 + 3 d1 + 9 d2 + 27 (d3 + 3 d4); entry = sum_e (d_e - 1) x_e
+    float2 ab[9];
+#pragma unroll
+    for (int m = 0; m < 9; ++m) {
+      const float l0 = static_cast<float>(m % 3 - 1), l1 = static_cast<float>(m / 3 - 1);
+      ab[m] = __ffma2_rn(make_float2(l0, l0), xv[0], __fmul2_rn(make_float2(l1, l1), xv[1]));
+    }
+    for (int hi = ctid >> 6; hi < T::kHi; hi += kCT / 64) {
       const float l3 = static_cast<float>(hi % 3 - 1), l4 = static_cast<float>(hi / 3 - 1);
       const float2 q = __ffma2_rn(make_float2(l3, l3), xv[3], __fmul2_rn(make_float2(l4, l4), xv[4]));
-      float2 qc[3], ab[9];
 #pragma unroll
       for (int d2 = 0; d2 < 3; ++d2) {
         const float l = static_cast<float>(d2 - 1);
-        qc[d2] = __ffma2_rn(make_float2(l, l), xv[2], q);
-      }
+        const float2 qc = __ffma2_rn(make_float2(l, l), xv[2], q);
+        const uint32_t row0 = col + static_cast<uint32_t>(9 * d2 + 27 * hi) * 256u;
 #pragma unroll
-      for (int m = 0; m < 9; ++m) {
-        const float l0 = static_cast<float>(m % 3 - 1), l1 = static_cast<float>(m / 3 - 1);
-        ab[m] = __ffma2_rn(make_float2(l0, l0), xv[0], __fmul2_rn(make_float2(l1, l1), xv[1]));
+        for (int m = 0; m < 9; ++m) sts_f2(row0 + m * 256u, __fadd2_rn(qc, ab[m]));
       }
+    }
+    // byte values 243..255 never occur: zero rows keep them harmless
+    for (int i = ctid; i < 13 * 64; i += kCT) {
+      const int v = 243 + i / 64, c = i % 64;
+      sts_f2(tbase + (c >> 5) * kPage + static_cast<uint32_t>(v) * 256u + (c & 31) * 8,
+             make_float2(0.0f, 0.0f));
+    }
+  } else {
+    // v = lo + 16 hi; the low two digits come from lo & 3 and lo >> 2
+    float2 av[4], bv[4];
 #pragma unroll
-      for (int lo = 0; lo < 27; ++lo)
-        sts_f2(col + static_cast<uint32_t>(lo + 27 * hi) * 256u, __fadd2_rn(qc[lo / 9], ab[lo % 9]));
-    } else {
-      // v = lo + 16 hi; low two digits from lo & 3 and lo >> 2 (1-bit: bit pairs)
-      float2 qb[4], av[4];
+    for (int m = 0; m < 4; ++m) {
+      if (FMT == LBQ_SIGN1) {
+        const float l0 = (m & 1) ? 1.0f : -1.0f, l1 = (m & 2) ? 1.0f : -1.0f;
+        av[m] = __ffma2_rn(make_float2(l0, l0), xv[0], __fmul2_rn(make_float2(l1, l1), xv[1]));
+        bv[m] = __ffma2_rn(make_float2(l0, l0), xv[2], __fmul2_rn(make_float2(l1, l1), xv[3]));
+      } else {
+        const float l = static_cast<float>(m) - 1.5f;
+        av[m] = __fmul2_rn(make_float2(l, l), xv[0]);
+        bv[m] = __fmul2_rn(make_float2(l, l), xv[1]);
+      }
+    }
+    for (int hi = ctid >> 6; hi < T::kHi; hi += kCT / 64) {
       float2 q;
       if (FMT == LBQ_SIGN1) {
         q = make_float2(0.0f, 0.0f);
@@ -219,39 +289,24 @@ __device__ __forceinline__ void build_slice(const Args<FMT>& a, int64_t j, uint3
           const float l = ((hi >> e) & 1) ? 1.0f : -1.0f;
           q = __ffma2_rn(make_float2(l, l), xv[4 + e], q);
         }
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const float l0 = (m & 1) ? 1.0f : -1.0f, l1 = (m & 2) ? 1.0f : -1.0f;
-          av[m] = __ffma2_rn(make_float2(l0, l0), xv[0], __fmul2_rn(make_float2(l1, l1), xv[1]));
-          qb[m] = __ffma2_rn(make_float2(l0, l0), xv[2], __ffma2_rn(make_float2(l1, l1), xv[3], q));
-        }
       } else {
         const float l2 = static_cast<float>(hi & 3) - 1.5f, l3 = static_cast<float>(hi >> 2) - 1.5f;
         q = __ffma2_rn(make_float2(l2, l2), xv[2], __fmul2_rn(make_float2(l3, l3), xv[3]));
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const float l = static_cast<float>(m) - 1.5f;
-          av[m] = __fmul2_rn(make_float2(l, l), xv[0]);
-          qb[m] = __ffma2_rn(make_float2(l, l), xv[1], q);
-        }
       }
 #pragma unroll
-      for (int lo = 0; lo < 16; ++lo)
-        sts_f2(col + static_cast<uint32_t>(lo + 16 * hi) * 256u, __fadd2_rn(qb[lo >> 2], av[lo & 3]));
+      for (int m1 = 0; m1 < 4; ++m1) {
+        const float2 qb = __fadd2_rn(q, bv[m1]);
+        const uint32_t row0 = col + static_cast<uint32_t>(4 * m1 + 16 * hi) * 256u;
+#pragma unroll
+        for (int m0 = 0; m0 < 4; ++m0) sts_f2(row0 + m0 * 256u, __fadd2_rn(qb, av[m0]));
+      }
     }
   }
-  if (FMT == LBQ_TERN5) {  // byte values 243..255 never occur: zero rows keep them harmless
-    for (int i = ctid; i < 13 * 64; i += 32 * kConsumers) {
-      const int v = 243 + i / 64, c = i % 64;
-      sts_f2(tbase + (c >> 5) * kPage + static_cast<uint32_t>(v) * 256u + (c & 31) * 8,
-             make_float2(0.0f, 0.0f));
-    }
-  }
-  named_bar_sync(1, 32 * kConsumers);
+  named_bar_sync(1, kCT);
 }
 
 template <int FMT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kMaxThreads, 1)
     gemv_lut_kernel(const __grid_constant__ CUtensorMap tm_codes,
                     const __grid_constant__ CUtensorMap tm_scales, const Args<FMT> a) {
   using T = Traits<FMT>;
@@ -259,13 +314,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_launch_dependents();
 
+  constexpr int kStages = T::kStages;
+  constexpr uint32_t kStageBytes = T::kStageBytes, kStageCodes = T::kStageCodes;
+  constexpr int kConsumers = T::kConsumers;
+  static_assert(kStages <= kMaxStages && kStages > kConsumers && kConsumers <= kMaxConsumers,
+                "stage ring");
   const uint32_t sbase = smem_u32(smem);
   const uint32_t tbase = (sbase + kPage - 1) & ~(kPage - 1);
   const uint32_t n_low = (tbase - sbase) / kStageBytes < kStages ? (tbase - sbase) / kStageBytes
                                                                  : kStages;
   const uint32_t high = tbase + 2 * kPage;  // first byte above the table
   const uint32_t tail = high + (kStages - n_low) * kStageBytes;
-  if (tail + kTailBytes > sbase + kSmem) {  // cannot happen with a 0 or 1 KB reserved prefix
+  if (tail + kTailBytes > sbase + T::kSmem) {  // cannot happen with a 0 or 1 KB reserved prefix
     if (tid == 0) atomicExch(a.fault, kFaultLayout);
     return;
   }
@@ -276,16 +336,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* xs = reinterpret_cast<float*>(smem + (tail - sbase));
   const uint32_t full0 = tail + 4096, empty0 = full0 + kStages * 8;
 
-  const int64_t NC = (a.N + kRows - 1) / kRows;
-  const int64_t U = static_cast<int64_t>(a.KS) * NC;
-  const int64_t u0 = static_cast<int64_t>(blockIdx.x) * U / gridDim.x;
-  const int64_t u1 = static_cast<int64_t>(blockIdx.x + 1) * U / gridDim.x;
+  // This CTA: slice j, 32-row chunks [c_lo, c_hi) of it (a.G CTAs share a slice).
+  const int32_t NC = static_cast<int32_t>((a.N + kRows - 1) / kRows);
+  const int32_t j = static_cast<int32_t>(blockIdx.x) / a.G;
+  const int32_t gs = static_cast<int32_t>(blockIdx.x) - j * a.G;
+  // (32-bit arithmetic: NC <= 16384 and G <= the SM count, so gs * NC fits; a 64-bit
+  // division here costs the kernel most of a microsecond)
+  const int32_t c_lo = static_cast<int32_t>(static_cast<uint32_t>(gs * NC) / static_cast<uint32_t>(a.G));
+  const int32_t c_hi =
+      static_cast<int32_t>(static_cast<uint32_t>((gs + 1) * NC) / static_cast<uint32_t>(a.G));
+  const int32_t n_units = c_hi - c_lo;
 
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 1);
-    }
+  if (tid < kStages) {  // one barrier pair per thread; each initialiser fences its own inits
+    mbar_init(full0 + 8 * tid, 1);
+    mbar_init(empty0 + 8 * tid, 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -296,26 +360,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_codes);
       if (T::kScaleBox) prefetch_tmap(&tm_scales);
       const uint32_t bytes = T::kPitch * kRows + T::kScaleBox * 2 * kRows;
-      int64_t issued = 0;
-      for (int64_t k = 0; k < u1 - u0; ++k) {
-        const int s = static_cast<int>(k % kStages);
-        const uint32_t use = static_cast<uint32_t>(k / kStages);
-        if (!mbar_wait(empty0 + 8 * s, (use & 1) ^ 1, a.fault, kFaultProducer)) break;
+      int32_t issued = 0;
+      int s = 0;
+      uint32_t phase = 0;
+      for (int32_t c = c_lo; c < c_hi; ++c) {
+        if (!mbar_wait(empty0 + 8 * s, phase ^ 1, a.fault, kFaultProducer)) break;
         ++issued;
-        const int64_t u = u0 + k, j = u / NC, c = u % NC;
         mbar_arrive_expect_tx(full0 + 8 * s, bytes);
         const uint32_t dst = stage_addr(s);
-        tma_load_2d(dst, &tm_codes, static_cast<int32_t>(j * T::kPitch),
-                    static_cast<int32_t>(c * kRows), full0 + 8 * s);
+        tma_load_2d(dst, &tm_codes, j * T::kPitch, c * kRows, full0 + 8 * s);
         if (T::kScaleBox)
-          tma_load_2d(dst + kStageCodes, &tm_scales, static_cast<int32_t>(j * T::kScaleBox),
-                      static_cast<int32_t>(c * kRows), full0 + 8 * s);
+          tma_load_2d(dst + kStageCodes, &tm_scales, j * T::kScaleBox, c * kRows, full0 + 8 * s);
+        if (++s == kStages) {
+          s = 0;
+          phase ^= 1;
+        }
       }
       // Before this lane exits, every copy it issued must have landed (normally the
       // consumers have already seen them all; this matters only after a fault).
-      for (int s = 0; s < kStages && s < issued; ++s) {
-        const int64_t k_last = s + (issued - 1 - s) / kStages * kStages;
-        mbar_wait(full0 + 8 * s, static_cast<uint32_t>(k_last / kStages) & 1, a.fault,
+      for (int s2 = 0; s2 < kStages && s2 < issued; ++s2) {
+        const int32_t k_last = s2 + (issued - 1 - s2) / kStages * kStages;
+        mbar_wait(full0 + 8 * s2, static_cast<uint32_t>(k_last / kStages) & 1, a.fault,
                   kFaultProducer, /*give_up_after_fault=*/false);
       }
     }
@@ -335,84 +400,85 @@ __global__ void __launch_bounds__(kThreads, 1)
       FMT == LBQ_TERN5 ? static_cast<uint32_t>(T::kPitch * lane + 28 * (lane / 7 < 3 ? lane / 7 : 3) + 26)
                        : static_cast<uint32_t>(kStageCodes + kSPitch * lane +
                                                2 * (lane / (FMT == LBQ_SIGN1 ? 4 : 2)));
-  bool ok = true;
+  build_slice<FMT>(a, j, tbase, xs, tid);
 
-  for (int64_t j = u0 / NC; j * NC < u1; ++j) {
-    named_bar_sync(1, 32 * kConsumers);  // every consumer is done with the previous table
-    build_slice<FMT>(a, j, tbase, xs, tid);
-    const int64_t kb = (u0 > j * NC ? u0 : j * NC) - u0;
-    const int64_t ke = ((j + 1) * NC < u1 ? (j + 1) * NC : u1) - u0;
-    int64_t k = kb + ((warp - kb) % kConsumers + kConsumers) % kConsumers;
-    for (; k < ke; k += kConsumers) {
-      const int s = static_cast<int>(k % kStages);
-      const uint32_t use = static_cast<uint32_t>(k / kStages);
-      const uint32_t stage = stage_addr(s);
-      const int64_t c = u0 + k - j * NC;
-      float acc[kRows];
-      if (ok) ok = mbar_wait(full0 + 8 * s, use & 1, a.fault, kFaultConsumer);
-      if (ok) {
-        uint32_t wa = stage + w_off, sa = stage + s_off;
-        // Gray-code walk over g; row (g ^ lane); two rows per step pair
+  bool ok = true;
+  // this warp's units: k = warp, warp + kConsumers, ... (stage k % kStages)
+  for (int32_t k = warp; k < n_units; k += kConsumers) {
+    const int s = k % kStages;
+    const uint32_t use = static_cast<uint32_t>(k / kStages);
+    const uint32_t stage = stage_addr(s);
+    float acc[kRows];
+    if (ok) ok = mbar_wait(full0 + 8 * s, use & 1, a.fault, kFaultConsumer);
+    if (ok) {
+      uint32_t wa = stage + w_off, sa = stage + s_off;
+      // Gray-code walk over g; row (g ^ lane); two rows per step pair
 #pragma unroll
-        for (int t = 0; t < kRows; t += 2) {
-          const int g0 = t ^ (t >> 1), g1 = (t + 1) ^ ((t + 1) >> 1);
-          const uint32_t wd0 = lds_u32(wa), sc0 = lds_u16(sa);
-          // step t -> t+1 flips bit 0 of g
-          const int sg0 = (g0 & 1) ? -1 : 1;
-          const uint32_t wa1 = wa + sg0 * dw.at(0), sa1 = sa + sg0 * ds.at(0);
-          const uint32_t wd1 = lds_u32(wa1), sc1 = lds_u16(sa1);
-          float a0, b0, a1, b1;
-          lookup4(wd0, lanereg, a0, b0);
-          lookup4(wd1, lanereg, a1, b1);
-          const float2 p = __fadd2_rn(make_float2(a0, a1), make_float2(b0, b1));
-          const float2 sc = make_float2(f16_bits_to_f32(sc0), f16_bits_to_f32(sc1));
-          const float2 r = __fmul2_rn(p, sc);
-          acc[g0] = r.x;
-          acc[g1] = r.y;
-          if (t + 2 < kRows) {  // step t+1 -> t+2 flips bit ctz(t+2) of g
-            const int b = __ffs(t + 2) - 1;
-            const int sg = ((g1 >> b) & 1) ? -1 : 1;
-            wa = wa1 + sg * dw.at(b);
-            sa = sa1 + sg * ds.at(b);
-          }
+      for (int t = 0; t < kRows; t += 2) {
+        const int g0 = t ^ (t >> 1), g1 = (t + 1) ^ ((t + 1) >> 1);
+        const uint32_t wd0 = lds_u32(wa), sc0 = lds_u16(sa);
+        // step t -> t+1 flips bit 0 of g
+        const int sg0 = (g0 & 1) ? -1 : 1;
+        const uint32_t wa1 = wa + sg0 * dw.at(0), sa1 = sa + sg0 * ds.at(0);
+        const uint32_t wd1 = lds_u32(wa1), sc1 = lds_u16(sa1);
+        const float2 p = lookup4x2(wd0, wd1, lanereg);
+        const float2 sc = make_float2(f16_bits_to_f32(sc0), f16_bits_to_f32(sc1));
+        const float2 r = __fmul2_rn(p, sc);
+        acc[g0] = r.x;
+        acc[g1] = r.y;
+        if (t + 2 < kRows) {  // step t+1 -> t+2 flips bit ctz(t+2) of g
+          const int b = __ffs(t + 2) - 1;
+          const int sg = ((g1 >> b) & 1) ? -1 : 1;
+          wa = wa1 + sg * dw.at(b);
+          sa = sa1 + sg * ds.at(b);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty0 + 8 * s);
-      } else {
-#pragma unroll
-        for (int i = 0; i < kRows; ++i) acc[i] = 0.0f;
       }
-      // butterfly: acc[i] holds row (i ^ lane); after it, acc[0] is row `lane`
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) {
-#pragma unroll
-        for (int i = 0; i < o; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i + o], o);
-      }
-      if (!ok) continue;
-      const float v = acc[0];
-      const int64_t r = c * kRows + lane;
-      if (a.KS == 1) {
-        if (r < a.N) a.y[r] = f32_to_bf16_bits(v);
-        continue;
-      }
-      if (r < a.N) a.part[j * a.N + r] = v;
-      __threadfence();
       __syncwarp();
-      unsigned last = 0;
-      if (lane == 0) last = (atomicAdd(a.cnt + c, 1u) == static_cast<unsigned>(a.KS - 1));
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {  // every slice of this chunk is in: sum them in slice order
-        __threadfence();
-        if (r < a.N) {
-          float sum = 0.0f;
-          for (int jj = 0; jj < a.KS; ++jj)
-            sum += __ldcg(a.part + static_cast<int64_t>(jj) * a.N + r);
-          a.y[r] = f32_to_bf16_bits(sum);
-        }
-        if (lane == 0) a.cnt[c] = 0u;
-      }
+      if (lane == 0) mbar_arrive(empty0 + 8 * s);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kRows; ++i) acc[i] = 0.0f;
+    }
+    // butterfly: acc[i] holds row (i ^ lane); after it, acc[0] is row `lane`
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+#pragma unroll
+      for (int i = 0; i < o; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i + o], o);
+    }
+    if (!ok) continue;
+    const int64_t r = static_cast<int64_t>(c_lo + k) * kRows + lane;
+    if (r < a.N) {
+      if (a.KS == 1)
+        a.y[r] = f32_to_bf16_bits(acc[0]);
+      else
+        a.part[static_cast<int64_t>(j) * a.N + r] = acc[0];
     }
   }
+}
+
+// Sums the slice sums of every row in slice order and writes bf16 y. Launched right
+// after the main kernel with programmatic dependent launch: it may start while that
+// kernel is finishing and waits for its results before reading them.
+__global__ void __launch_bounds__(256) splitk_sum_kernel(const float* __restrict__ part, int KS,
+                                                         int64_t N, uint16_t* __restrict__ y) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (r >= N) return;
+  const float* pr = part + r;
+  float sum = 0.0f;
+  // all of a row's loads are issued before the sum (16 slices per round); the
+  // additions then run in slice order
+  for (int j = 0; j < KS; j += 16) {
+    float v[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+      v[q] = j + q < KS ? __ldcg(pr + static_cast<int64_t>(j + q) * N) : 0.0f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+      if (j + q < KS) sum += v[q];
+  }
+  y[r] = f32_to_bf16_bits(sum);
 }
 
 // The device word the kernels' bounded waits report to (one per device).
@@ -460,7 +526,7 @@ cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uin
   if (dev >= 0 && dev < 64 && !configured[dev]) {
     cudaError_t e = cudaFuncSetAttribute(gemv_lut_kernel<FMT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmem));
+                                         static_cast<int>(T::kSmem));
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
@@ -474,7 +540,6 @@ cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uin
   a.nblk = static_cast<int>(w->K / (FMT == LBQ_Q2RHT ? kQ2Block : kTernBlock));
   a.fault = lbq_fault_word();
   if (!a.fault) return cudaErrorInvalidDevicePointer;
-  a.cnt = static_cast<uint32_t*>(ws);
   a.part = ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + kWsCounterBytes) : nullptr;
 
   CUtensorMap tc, ts;
@@ -492,20 +557,29 @@ cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uin
     ts = tc;  // unused
   }
   const int64_t NC = (w->N + kRows - 1) / kRows;
-  const int64_t units = static_cast<int64_t>(a.KS) * NC;
-  const int64_t grid = units < sm_count() ? units : sm_count();
+  // Each CTA works on one slice only (one table build): floor(SMs / KS) CTAs per slice.
+  const int64_t per = sm_count() / a.KS > 1 ? sm_count() / a.KS : 1;
+  a.G = static_cast<int>(per < NC ? per : NC);
+  const int64_t grid = static_cast<int64_t>(a.KS) * a.G;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmem;
+  cfg.blockDim = dim3(32 * (T::kConsumers + 1));
+  cfg.dynamicSmemBytes = T::kSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_lut_kernel<FMT>, tc, ts, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_lut_kernel<FMT>, tc, ts, a);
+  if (e != cudaSuccess || a.KS == 1) return e;
+  cudaLaunchConfig_t cfg2 = cfg;
+  cfg2.gridDim = dim3(static_cast<unsigned>((w->N + 255) / 256));
+  cfg2.blockDim = dim3(256);
+  cfg2.dynamicSmemBytes = 0;
+  return cudaLaunchKernelEx(&cfg2, splitk_sum_kernel, static_cast<const float*>(a.part), a.KS,
+                            static_cast<int64_t>(w->N), y);
 }
 
 }  // namespace
