@@ -2,8 +2,10 @@
 //
 // Same formats and rules as gemv.cu (ternary add/subtract/skip per block,
 // pptc.cn §1.2 and mhpq.cn §2.1-2.2; 1-bit Q1_0, neodrop.ai part 2; 2-bit with the
-// rotated input, feinterview.poetries.top). This file holds the straightforward
-// kernel: one warp per (row, group of activation rows), blocks decoded in registers.
+// rotated input, feinterview.poetries.top). The ternary format goes to the tensor-core
+// kernel in gemm_tc.cu; this file holds the straightforward kernel the 1-bit and
+// 2-bit formats use for now: one warp per (row, group of activation rows), blocks
+// decoded in registers.
 #include "lbq_common.cuh"
 
 namespace {
@@ -94,6 +96,7 @@ __global__ void __launch_bounds__(256) gemm_rowwarp(const uint8_t* __restrict__ 
 }  // namespace
 
 size_t lbq_gemm_workspace(const lbq_weights* w, int64_t M) {
+  if (w->fmt == LBQ_TERN5) return lbq_gemm_tc_workspace(w, M);
   return w->fmt == LBQ_Q2RHT
              ? kWsCounterBytes + static_cast<size_t>(w->K) * static_cast<size_t>(M) * sizeof(float)
              : 0;
@@ -108,10 +111,8 @@ cudaError_t lbq_launch_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, 
   const uint8_t* codes = static_cast<const uint8_t*>(w->codes);
   const uint16_t* scales = static_cast<const uint16_t*>(w->scales);
   switch (w->fmt) {
-    case LBQ_TERN5:
-      gemm_rowwarp<LBQ_TERN5><<<grid, 32 * warps, 0, s>>>(codes, w->code_stride, nullptr, 0, w->K,
-                                                          w->N, X, nullptr, M, m_per_cta, Y);
-      break;
+    case LBQ_TERN5:  // tensor-core path (gemm_tc.cu)
+      return lbq_launch_gemm_tc(w, X, M, Y, ws, s);
     case LBQ_SIGN1:
       gemm_rowwarp<LBQ_SIGN1><<<grid, 32 * warps, 0, s>>>(
           codes, w->code_stride, scales, w->scale_stride, w->K, w->N, X, nullptr, M, m_per_cta, Y);

@@ -105,5 +105,8 @@ unsigned* lbq_fault_word();
 cudaError_t lbq_launch_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D,
                             uint16_t* y, void* ws, cudaStream_t s);
 size_t lbq_gemm_workspace(const lbq_weights* w, int64_t M);
+size_t lbq_gemm_tc_workspace(const lbq_weights* w, int64_t M);
+cudaError_t lbq_launch_gemm_tc(const lbq_weights* w, const uint16_t* X, int64_t M, uint16_t* Y,
+                               void* ws, cudaStream_t s);
 cudaError_t lbq_launch_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const int8_t* D,
                             uint16_t* Y, void* ws, cudaStream_t s);

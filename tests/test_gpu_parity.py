@@ -258,3 +258,41 @@ def test_no_bounded_device_wait_gave_up(L):
     """After every product above, no in-kernel wait ran out (the fault record is clear)."""
     torch.cuda.synchronize()
     assert L.lbq_device_fault() == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 1024), (3, 130, 640), (16, 128, 128), (128, 384, 1024),
+                                   (512, 256, 5120), (200, 1000, 2048)])
+def test_ternary_gemm_tensor_cores(L, orc, M, N, K):
+    """The tensor-core ternary product: ragged M and N, K from one block to 40."""
+    W = synth.weights(N, K, 6000 + M + N)
+    X = synth.activations(M, K, 7000 + M)
+    pw, codes, scales = _pack_both(L, orc, TERN5, W)
+    Yg = L.lbq_gemm(pw, X.cuda())
+    Y, B = orc.gemm(TERN5, codes, scales, K, synth.bf16_bits(X), None, nthreads=NTHREADS)
+    _check_products(Yg, Y, B, f"tern gemm M={M} N={N} K={K}")
+
+
+def test_ternary_gemm_large_activations_are_scaled_into_fp16(L, orc):
+    """Rows of X beyond fp16's range (bf16 values up to 3e38 are finite) still come out right."""
+    M, N, K = 4, 128, 512
+    W = synth.weights(N, K, 61)
+    X = synth.activations(M, K, 62)
+    X[1] *= 2.0 ** 40
+    X[2] *= 2.0 ** -30
+    pw, codes, scales = _pack_both(L, orc, TERN5, W)
+    Yg = L.lbq_gemm(pw, X.cuda())
+    Y, B = orc.gemm(TERN5, codes, scales, K, synth.bf16_bits(X), None)
+    _check_products(Yg, Y, B, "scaled rows")
+
+
+def test_ternary_gemm_27b_gate_up_sampled(L, orc):
+    """M = 512 tokens through a full 27B gate+up matrix; sampled rows checked exactly."""
+    N, K, M = 2 * synth.FFN, synth.HIDDEN, 512
+    Wd = synth.weights(N, K, 777, device="cuda")
+    pw = L.lbq_pack(TERN5, Wd)
+    X = synth.activations(M, K, 778, device="cuda")
+    Yg = L.lbq_gemm(pw, X)
+    rows = torch.tensor([0, 5, 127, 128, 9999, N - 129, N - 1], device="cuda")
+    codes, scales = orc.pack(TERN5, Wd[rows].cpu().numpy())
+    Y, B = orc.gemm(TERN5, codes, scales, K, synth.bf16_bits(X), None, nthreads=NTHREADS)
+    _check_products(Yg[:, rows], Y, B, "27B gate+up, M=512")
