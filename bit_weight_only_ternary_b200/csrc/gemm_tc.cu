@@ -18,14 +18,20 @@
 // memory; activations: fp16 in shared memory. Warp roles:
 //   warp 0   one lane streams fp16 activation tiles with 2D TMA (128-byte swizzle)
 //   warp 1   allocates tensor memory; one lane issues the MMAs and commits stages
-//   warps 4-11 two threads per weight row, one per 64-weight half of each block:
-//            packed words arrive with cp.async (4 blocks in flight), each byte
-//            becomes five fp16 trits through small tables, is scaled, and the 64
-//            fp16 go straight to tensor memory (tcgen05.st: the weight operand is
-//            read by the MMA from tensor memory, so neither the stores nor the
-//            MMA's operand reads use shared-memory bandwidth); then the same warps
-//            read the accumulator (warp w reads lane quarter w % 4, the two warp
-//            groups split the columns) and write bf16 Y.
+//   warp 2   one lane streams the packed weight rows with 2D TMA, four blocks
+//            (112 bytes) of 128 rows per copy
+//   warps 4-19 four threads per weight row, one per 32-weight quarter of each block.
+//            Each byte becomes five fp16 values through one lookup: a table in
+//            shared memory maps the byte to the byte-permute selectors that pick
+//            +s, -s or 0 out of a register holding the block's scale, so a byte
+//            costs one table load (its address is itself one byte permute of the
+//            packed word) and one permute per pair of weights. The table is
+//            replicated for the 16 lanes of a half warp, so the lookups of a warp
+//            never collide on a bank. The 32 fp16 go straight to tensor memory
+//            (tcgen05.st: the MMA reads the weight operand from tensor memory;
+//            a block's store completes while the next block is decoded); then the
+//            same warps read the accumulator (warp w reads lane quarter w % 4, the
+//            four warp groups split the columns) and write bf16 Y.
 // Every wait is bounded (see sm100_async.cuh).
 #include <cudaTypedefs.h>
 
@@ -36,35 +42,46 @@ namespace {
 using namespace lbq;
 
 constexpr int kTileN = 128;     // weight rows per tile (MMA M)
-constexpr int kTileK = 128;     // K per stage
+constexpr int kTileK = 128;     // K per stage (one ternary block)
 constexpr int kMaxTileM = 128;  // tokens per tile (MMA N)
-constexpr int kStagesTC = 3;
-constexpr int kRawDepth = 4;    // packed blocks in flight per decoder thread
-constexpr int kDecoders = 2 * kTileN;  // two threads per weight row
+constexpr int kStagesTC = 4;
+constexpr int kDecoders = 4 * kTileN;  // four threads per weight row, a quarter block each
 constexpr int kThreadsTC = 128 + kDecoders;
-constexpr uint32_t kStageB = 2 * kMaxTileM * 128;
-// Tensor memory (512 columns): the fp32 accumulator in columns [0, tile_m), the fp16
-// weight stages at kTmemA + 64 s (128 rows x 128 K = 64 columns each).
-constexpr uint32_t kTmemCols = 512, kTmemA = 256;
-constexpr uint32_t kOffB = 0;
-constexpr uint32_t kOffRaw = kOffB + kStagesTC * kStageB;
-constexpr uint32_t kRawWords = 5;  // words of a block a half-row decoder needs (see below)
-constexpr uint32_t kRawPerThread = kRawDepth * kRawWords * 4;
-constexpr uint32_t kOffLut = kOffRaw + kDecoders * kRawPerThread;
-constexpr uint32_t kLutBytes = 1024;  // the four small trit tables (see build_trit_tables)
-constexpr uint32_t kOffBar = (kOffLut + kLutBytes + 7) / 8 * 8;
-constexpr uint32_t kOffTmem = kOffBar + (3 * kStagesTC + 1) * 8;
-constexpr size_t kSmemTC = kOffTmem + 16 + 1024;  // + slack to align the base to 1024
-constexpr unsigned kFaultX = 4, kFaultMma = 5, kFaultDecode = 6, kFaultEpilogue = 7;
+constexpr int kChunkBlocks = 4;        // packed blocks per weight copy: 112 bytes, a multiple of 16
+constexpr uint32_t kChunkRowBytes = kChunkBlocks * kTernBlockBytes;
+constexpr uint32_t kRawStageBytes = kChunkRowBytes * kTileN;
+constexpr int kRawStages = 2;
+constexpr uint32_t kStageB = 2 * kMaxTileM * 128;  // two 64-k slabs of activations
+// Tensor memory (512 columns): nacc fp32 accumulators of tile_m columns each in
+// [0, 256), the fp16 weight stages at kTmemA + 64 s (128 rows x 128 K = 64 columns
+// each). Successive MMAs go to different accumulators: an MMA that depends on the
+// previous one's accumulator waits for it to finish, and a K = 16 step with a small
+// token count is far shorter than that latency.
+constexpr uint32_t kTmemCols = 512, kTmemA = 256, kAccCols = 256;
+// Shared memory. The selector table sits at a 64 KB-aligned shared-window address T
+// so that a table address is T | byte << 8 | lane slot (one byte permute):
+//   [T - kLowBytes, T)   mbarriers + TMEM slot (256 B), raw weight ring, activation stage 0
+//   [T, T + 62208)        selector table: [byte 0..242][even/odd][16 lanes] x 8 bytes
+//   [T + 0xF400, ...)     activation stages 1..3
+// The dynamic window starts 1 KB into shared memory on sm_100 (T = 64 KB); the
+// kernel checks the placement and reports a fault rather than run off its end.
+constexpr uint32_t kTabBytes = 243 * 256;
+constexpr uint32_t kLowBytes = 256 + kRawStages * kRawStageBytes + kStageB;
+constexpr uint32_t kHighB = 0xF400;  // first activation stage above the table (1 KB aligned)
+constexpr uint32_t kHighBytes = kHighB + (kStagesTC - 1) * kStageB;
+constexpr size_t kSmemTC = 0x10000 - 0x400 + kHighBytes;
+static_assert(kTabBytes <= kHighB, "table overlaps stage 1");
+static_assert(0x400 + kLowBytes <= 0x10000, "low region does not fit below 64 KB");
+static_assert(kSmemTC <= 232448, "over the shared-memory limit");
+constexpr unsigned kFaultX = 4, kFaultMma = 5, kFaultDecode = 6, kFaultEpilogue = 7, kFaultW = 8,
+                   kFaultSmem = 9;
 
 struct TcArgs {
-  const uint8_t* codes;
-  int64_t cstride;
   int64_t K, N, M;
   const int* xexp;  // token row m of X was scaled by 2^-xexp[m]
   uint16_t* Y;
   int tile_m;       // MMA N: tokens per tile
-  uint32_t tmem_cols;
+  int nacc;         // independent accumulators (a power of two, nacc * tile_m <= 256)
   int kb_per_split; // K blocks per CTA along grid z (split-K)
   float* part;      // [splits][M][N] fp32 partial products, or null (no split)
   unsigned* fault;
@@ -93,109 +110,161 @@ __device__ __forceinline__ uint4 lds_u128(uint32_t addr) {
                : "r"(addr));
   return v;
 }
-__device__ __forceinline__ void sts_u128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                         uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
+// ---------------------------------------------------------------- byte -> fp16 values
+// A byte v = d0 + 3 d1 + 9 d2 + 27 d3 + 81 d4 holds five digits d = t + 1 (weights
+// 5j .. 5j + 4 of the block for byte j). A register V = (s, -s) as two fp16, next
+// to a zero register, lets one byte permute build a pair of fp16 weights: the
+// selector code of a digit names the two bytes of +s (digit 2), -s (0) or zero (1).
+constexpr uint32_t sel_code(uint32_t d) { return d == 2 ? 0x10u : (d == 0 ? 0x32u : 0x54u); }
+constexpr uint32_t digit(uint32_t v, int i) {
+  return i == 0 ? v % 3 : (i == 1 ? v / 3 % 3 : (i == 2 ? v / 9 % 3 : (i == 3 ? v / 27 % 3 : v / 81)));
 }
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
+// Byte j's first weight is the low half of a pair when j is even (5j even):
+//   even entry: x = codes of (t0, t1, t2, t3), y = code of t4 (low half of the next pair)
+//   odd entry:  x = code of t0 in the high half, y = codes of (t1, t2, t3, t4)
+// so an even byte gives pairs (t0,t1) = x, (t2,t3) = x >> 16, and with the odd byte
+// after it (t4, u0) = y_even | x_odd, (u1,u2) = y_odd, (u3,u4) = y_odd >> 16.
+struct SelTable {
+  uint32_t w[243][2][2];
+};
+constexpr SelTable make_sel_table() {
+  SelTable t{};
+  for (uint32_t v = 0; v < 243; ++v) {
+    uint32_t c[5] = {};
+    for (int i = 0; i < 5; ++i) c[i] = sel_code(digit(v, i));
+    t.w[v][0][0] = c[0] | c[1] << 8 | c[2] << 16 | c[3] << 24;
+    t.w[v][0][1] = c[4];
+    t.w[v][1][0] = c[0] << 8;
+    t.w[v][1][1] = c[1] | c[2] << 8 | c[3] << 16 | c[4] << 24;
+  }
+  return t;
 }
+__device__ const SelTable g_sel_table = make_sel_table();
 
-// A ternary byte v = lo + 27 hi (lo < 27 holds trits 0..2, hi < 9 trits 3..4; hi is
-// (v * 1214) >> 15, exact for every byte value) decodes through four small tables of
-// fp16 trits (-1, 0, +1), one pair per word, for the two word alignments a byte's
-// five weights can take (5 j is even for even j):
-//   even: lo -> {(t0, t1), (t2, 0)} at +0     hi -> {(0, t3), (t4, 0)} at +512
-//   odd:  lo -> {(0, t0), (t1, t2)} at +256   hi -> (t3, t4)           at +640
-// A few hundred bytes, so the warps' random lookups rarely collide on a bank.
-constexpr uint32_t kT27e = 0, kT27o = 256, kT9e = 512, kT9o = 640;
-
-__device__ __forceinline__ uint32_t trit_f16(int d) {  // digit 0, 1, 2 -> fp16 -1, 0, +1
-  return d == 0 ? 0xBC00u : (d == 1 ? 0u : 0x3C00u);
-}
-
-__device__ __forceinline__ void build_trit_tables(uint32_t lut, int tid) {
-  if (tid < 27) {
-    const uint32_t t0 = trit_f16(tid % 3), t1 = trit_f16(tid / 3 % 3), t2 = trit_f16(tid / 9);
-    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(lut + kT27e + 8u * tid), "r"(t0 | (t1 << 16)),
-                 "r"(t2)
-                 : "memory");
-    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(lut + kT27o + 8u * tid), "r"(t0 << 16),
-                 "r"(t1 | (t2 << 16))
-                 : "memory");
-  } else if (tid >= 32 && tid < 41) {
-    const int h = tid - 32;
-    const uint32_t t3 = trit_f16(h % 3), t4 = trit_f16(h / 3);
-    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(lut + kT9e + 8u * h), "r"(t3 << 16), "r"(t4)
-                 : "memory");
-    asm volatile("st.shared.b32 [%0], %1;" ::"r"(lut + kT9o + 4u * h), "r"(t3 | (t4 << 16)) : "memory");
+// Replicates the table into shared memory as [byte][even/odd][16 lane slots] x 8 bytes.
+__device__ __forceinline__ void load_sel_table(uint32_t tab, int tid) {
+  const uint2* src = reinterpret_cast<const uint2*>(&g_sel_table);
+  constexpr int kSlots = 243 * 2 * 16;
+#pragma unroll 4
+  for (int i = tid; i < kSlots; i += kThreadsTC) {
+    const uint2 e = __ldg(src + (i >> 4));
+    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(tab + 8u * i), "r"(e.x), "r"(e.y) : "memory");
   }
 }
 
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   uint2 v;
   asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
 }
 
-// Places byte j's five fp16 trits into hv (pair index b0 = the pair holding weight
-// 5j, relative to hv[0]); pairs outside [0, kPairs) are skipped.
-template <int kPairs>
-__device__ __forceinline__ void place_byte(uint32_t (&hv)[kPairs], int j, int b0, uint32_t v,
-                                           uint32_t lut) {
-  const uint32_t hi = (v * 1214u) >> 15, lo = v - 27u * hi;
-  if (!(j & 1)) {
-    const uint2 a = lds64(lut + kT27e + 8u * lo), c = lds64(lut + kT9e + 8u * hi);
-    if (b0 >= 0 && b0 < kPairs) hv[b0] = a.x;
-    if (b0 + 1 >= 0 && b0 + 1 < kPairs) hv[b0 + 1] = a.y | c.x;
-    if (b0 + 2 >= 0 && b0 + 2 < kPairs) hv[b0 + 2] = c.y;
-  } else {
-    const uint2 a = lds64(lut + kT27o + 8u * lo);
-    const uint32_t c = lds32(lut + kT9o + 4u * hi);
-    if (b0 >= 0 && b0 < kPairs) hv[b0] |= a.x;
-    if (b0 + 1 >= 0 && b0 + 1 < kPairs) hv[b0 + 1] = a.y;
-    if (b0 + 2 >= 0 && b0 + 2 < kPairs) hv[b0 + 2] = c;
+// Word i of the block b of a 4-block row chunk held in raw[7] (compile-time indices).
+template <int kB, int kI>
+__device__ __forceinline__ uint32_t raw_word(const uint4 (&raw)[7]) {
+  constexpr int w = 7 * kB + kI;
+  const uint4 q = raw[w >> 2];
+  return (w & 3) == 0 ? q.x : ((w & 3) == 1 ? q.y : ((w & 3) == 2 ? q.z : q.w));
+}
+
+// Decodes bytes [kJ, kJ1] of block kB into pairs hv[p - kP0] (pairs outside
+// [kP0, kP0 + 16) are skipped). base_e / base_o: the table address of byte 0 for this
+// lane (even / odd entries); V: (s, -s).
+template <int kB, int kJ, int kJ1, int kP0>
+struct DecodeBytes {
+  static __device__ __forceinline__ void run(const uint4 (&raw)[7], uint32_t base_e, uint32_t base_o,
+                                             uint32_t V, uint32_t carry, uint32_t (&hv)[16]) {
+    const uint32_t word = raw_word<kB, kJ / 4>(raw);
+    constexpr uint32_t sel = 0x7604u | ((kJ & 3) << 4);  // lane slot, byte kJ & 3, table base
+    if constexpr ((kJ & 1) == 0) {
+      const uint2 e = lds64(prmt(word, base_e, sel));
+      constexpr int p = 5 * kJ / 2 - kP0;
+      if constexpr (p >= 0 && p < 16) hv[p] = prmt(V, 0u, e.x);
+      if constexpr (p + 1 >= 0 && p + 1 < 16) hv[p + 1] = prmt(V, 0u, e.x >> 16);
+      if constexpr (kJ < kJ1) carry = e.y;
+    } else {
+      const uint2 o = lds64(prmt(word, base_o, sel));
+      constexpr int p = (5 * kJ - 1) / 2 - kP0;
+      if constexpr (p >= 0 && p < 16) hv[p] = prmt(V, 0u, carry | o.x);
+      if constexpr (p + 1 >= 0 && p + 1 < 16) hv[p + 1] = prmt(V, 0u, o.y);
+      if constexpr (p + 2 >= 0 && p + 2 < 16) hv[p + 2] = prmt(V, 0u, o.y >> 16);
+    }
+    if constexpr (kJ < kJ1) DecodeBytes<kB, kJ + 1, kJ1, kP0>::run(raw, base_e, base_o, V, carry, hv);
+  }
+};
+
+// The 32 fp16 weights of quarter r of block kB of the chunk, in pairs (pairs 16 r ..
+// 16 r + 15 of the block). Quarter 0 = bytes 0..6, 1 = bytes 6..12, 2 = bytes 12..19,
+// 3 = bytes 19..25 (the bytes at the seams are decoded by both neighbours; byte 25's
+// last two digits are padding).
+template <int kB>
+__device__ __forceinline__ void decode_quarter(const uint4 (&raw)[7], int r, uint32_t base_e,
+                                               uint32_t base_o, uint32_t (&hv)[16]) {
+  const uint32_t sw = raw_word<kB, 6>(raw);              // bytes 24..27: scale in the high half
+  const uint32_t V = prmt(sw, sw ^ 0x80000000u, 0x7632u);  // (s, -s)
+  switch (r) {
+    case 0: DecodeBytes<kB, 0, 6, 0>::run(raw, base_e, base_o, V, 0u, hv); break;
+    case 1: DecodeBytes<kB, 6, 12, 16>::run(raw, base_e, base_o, V, 0u, hv); break;
+    case 2: DecodeBytes<kB, 12, 19, 32>::run(raw, base_e, base_o, V, 0u, hv); break;
+    default: DecodeBytes<kB, 19, kTernCodeBytes - 1, 48>::run(raw, base_e, base_o, V, 0u, hv); break;
   }
 }
 
 __global__ void __launch_bounds__(kThreadsTC, 1)
-    gemm_tern_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const TcArgs a) {
+    gemm_tern_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
+                        const __grid_constant__ CUtensorMap tm_w, const TcArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
-  const uint32_t s0 = (sraw + 1023u) & ~1023u;  // 1024-aligned: 128-byte swizzle atoms
+  const uint32_t tab = (sraw + kLowBytes + 0xFFFFu) & ~0xFFFFu;
+  if (tab - kLowBytes < sraw || tab + kHighBytes > sraw + static_cast<uint32_t>(kSmemTC)) {
+    if (threadIdx.x == 0) atomicExch(a.fault, kFaultSmem);  // placement assumption broken
+    return;
+  }
+  const uint32_t bstage0 = tab - kStageB;
+  const uint32_t rawring = bstage0 - kRawStages * kRawStageBytes;
+  const uint32_t bars = rawring - 256;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kTileN;
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * a.tile_m;
-  // this CTA's K blocks: [kb0, kb0 + nkb) (all of K unless split over grid z)
+  // this CTA's K blocks: [kb0, kb0 + nkb) (all of K unless split over grid z);
+  // kb_per_split is a multiple of the chunk
   const int kb0 = static_cast<int>(blockIdx.z) * a.kb_per_split;
   const int nkb_all = static_cast<int>(a.K / kTileK);
   const int nkb = (nkb_all - kb0 < a.kb_per_split) ? nkb_all - kb0 : a.kb_per_split;
-  const uint32_t fullA = s0 + kOffBar, fullB = fullA + 8 * kStagesTC;
+  const int nchunks = (nkb + kChunkBlocks - 1) / kChunkBlocks;
+  const uint32_t fullA = bars, fullB = fullA + 8 * kStagesTC;
   const uint32_t empty = fullB + 8 * kStagesTC, accum = empty + 8 * kStagesTC;
-  const uint32_t lut = s0 + kOffLut;
+  const uint32_t fullR = accum + 8, emptyR = fullR + 8 * kRawStages;
+  const uint32_t tslot = emptyR + 8 * kRawStages;
+  auto bstage = [&](int s) { return s == 0 ? bstage0 : tab + kHighB + (s - 1) * kStageB; };
 
-  build_trit_tables(lut, tid);
+  load_sel_table(tab, tid);
   if (tid == 0) {
     for (int s = 0; s < kStagesTC; ++s) {
       mbar_init(fullA + 8 * s, kDecoders);  // every decoder thread arrives
-      mbar_init(fullB + 8 * s, 1);       // the TMA lane arrives (+ bytes)
-      mbar_init(empty + 8 * s, 1);       // the MMA commit arrives
+      mbar_init(fullB + 8 * s, 1);          // the activation TMA lane arrives (+ bytes)
+      mbar_init(empty + 8 * s, 1);          // the MMA commit arrives
+    }
+    for (int r = 0; r < kRawStages; ++r) {
+      mbar_init(fullR + 8 * r, 1);          // the weight TMA lane arrives (+ bytes)
+      mbar_init(emptyR + 8 * r, kDecoders); // every decoder thread has read its row
     }
     mbar_init(accum, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(s0 + kOffTmem, kTmemCols);
+    tmem_alloc(tslot, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_raw + (s0 - sraw) + kOffTmem);
+  uint32_t tmem;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(tmem) : "r"(tslot));
 
   if (warp == 0) {
     // ---------------- activations: two 64-k boxes per stage, 128-byte swizzled
@@ -209,7 +278,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (!mbar_wait(empty + 8 * s, (use & 1) ^ 1, a.fault, kFaultX)) break;
         ++issued;
         mbar_arrive_expect_tx(fullB + 8 * s, bytes);
-        const uint32_t dst = s0 + kOffB + s * kStageB;
+        const uint32_t dst = bstage(s);
         tma_load_2d(dst, &tm_x, (kb0 + kb) * kTileK, static_cast<int32_t>(m0), fullB + 8 * s);
         tma_load_2d(dst + static_cast<uint32_t>(a.tile_m) * 128u, &tm_x, (kb0 + kb) * kTileK + 64,
                     static_cast<int32_t>(m0), fullB + 8 * s);
@@ -220,112 +289,124 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
                   a.fault, kFaultX, /*give_up_after_fault=*/false);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issue: 8 instructions of K = 16 per stage
-    if (lane == 0) {
-      const uint32_t idesc = idesc_f16_m128(a.tile_m);
-      const uint32_t slab_b = static_cast<uint32_t>(a.tile_m) * 128u;
+    // ---------------- MMA issue: 8 instructions of K = 16 per stage. The whole warp
+    // runs the loop (so descriptors stay warp-uniform); one elected lane issues.
+    const uint32_t idesc = idesc_f16_m128(a.tile_m);
+    const uint32_t slab_b = static_cast<uint32_t>(a.tile_m) * 128u;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % kStagesTC;
+      const uint32_t par = static_cast<uint32_t>(kb / kStagesTC) & 1;
       bool ok = true;
-      for (int kb = 0; kb < nkb && ok; ++kb) {
-        const int s = kb % kStagesTC;
-        const uint32_t par = static_cast<uint32_t>(kb / kStagesTC) & 1;
+      if (lane == 0)
         ok = mbar_wait(fullA + 8 * s, par, a.fault, kFaultMma) &&
              mbar_wait(fullB + 8 * s, par, a.fault, kFaultMma);
-        if (!ok) break;
-        tc_fence_after_sync();
-        const uint32_t ta = tmem + kTmemA + 64u * s, sb = s0 + kOffB + s * kStageB;
-#pragma unroll
-        for (int ks = 0; ks < kTileK / 16; ++ks) {  // K = 16: 8 tensor-memory columns of A
-          const uint32_t slab = ks >> 2, koff = (ks & 3) * 32;
-          mma_f16_ts(tmem, ta + 8u * ks, sw128_desc(sb + slab * slab_b + koff), idesc,
-                     (kb | ks) != 0 ? 1u : 0u);
-        }
-        mma_commit(empty + 8 * s);  // the stage is free once these MMAs are done
-      }
-      mma_commit(accum);  // the accumulator is complete once every MMA is done
-    }
-    __syncwarp();
-  } else if (warp >= 4) {
-    // ---------------- decode: thread d owns row d % 128, half h = d / 128 of each block.
-    // Half 0 = weights 0..63 = bytes 0..12 (byte 12 only up to its 4th trit); half 1 =
-    // weights 64..127 = byte 12's 5th trit and bytes 13..25. Half 0 copies words 0..3
-    // and 6 (the scale), half 1 words 3..6.
-    const int d = tid - 128;
-    const int row = d & (kTileN - 1), h = d >> 7;
-    const int64_t n = n0 + row;
-    const bool rv = n < a.N;
-    const uint32_t* src =
-        reinterpret_cast<const uint32_t*>(a.codes + (rv ? n : 0) * a.cstride) + 7 * kb0;
-    const uint32_t ring = s0 + kOffRaw + static_cast<uint32_t>(d) * kRawPerThread;
-    const int wsrc[kRawWords] = {h ? 3 : 0, h ? 4 : 1, h ? 5 : 2, h ? 6 : 3, 6};
-#pragma unroll 1
-    for (int p = 0; p < kRawDepth; ++p) {
-      if (rv && p < nkb)
-        for (int q = 0; q < kRawWords; ++q)
-          cp_async4(ring + (p * kRawWords + q) * 4, src + p * 7 + wsrc[q]);
-      cp_async_commit();
-    }
-    bool ok = true;
-#pragma unroll 1
-    for (int kb = 0; kb < nkb; ++kb) {
-      cp_async_wait<kRawDepth - 1>();  // block kb has landed in its ring slot
-      const uint32_t slot = ring + (kb % kRawDepth) * kRawWords * 4;
-      uint32_t w[kRawWords];
-#pragma unroll
-      for (int q = 0; q < kRawWords; ++q) w[q] = rv ? lds32(slot + 4 * q) : 0u;
-      if (rv && kb + kRawDepth < nkb)
-        for (int q = 0; q < kRawWords; ++q)
-          cp_async4(slot + 4 * q, src + (kb + kRawDepth) * 7 + wsrc[q]);
-      cp_async_commit();
-
-      uint32_t hv[32];  // this half's 64 fp16 weights, in pairs
-      if (h == 0) {
-        // bytes 0..12 = w[0..3]; byte j covers weights 5j..5j+4 (pair 5j/2)
-#pragma unroll
-        for (int j = 0; j < 13; ++j)
-          place_byte<32>(hv, j, (5 * j) >> 1, (w[j >> 2] >> (8 * (j & 3))) & 0xFFu, lut);
-      } else {
-        // w[0..3] = words 3..6 = bytes 12..27: byte 12 (the low byte of w[0]) gives
-        // weight 64 with its 5th trit; bytes 13..25 follow; pairs relative to weight 64
-#pragma unroll
-        for (int j = 12; j < kTernCodeBytes; ++j) {
-          const int jj = j - 12;
-          place_byte<32>(hv, j, ((5 * j) >> 1) - 32, (w[jj >> 2] >> (8 * (jj & 3))) & 0xFFu, lut);
-        }
-      }
-      const uint32_t sbits = (h ? w[3] : w[4]) >> 16;
-      const __half2 s2 = __halves2half2(__ushort_as_half(static_cast<uint16_t>(sbits)),
-                                        __ushort_as_half(static_cast<uint16_t>(sbits)));
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const __half2 t = *reinterpret_cast<const __half2*>(&hv[i]);
-        const __half2 p = __hmul2(t, s2);  // exact: t is -1, 0 or +1
-        hv[i] = *reinterpret_cast<const uint32_t*>(&p);
-      }
-
-      const int s = kb % kStagesTC;
-      const uint32_t use = static_cast<uint32_t>(kb / kStagesTC);
-      if (ok) ok = mbar_wait(empty + 8 * s, (use & 1) ^ 1, a.fault, kFaultDecode);
-      __syncwarp();  // tcgen05.st is warp-collective
+      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
       tc_fence_after_sync();
-      // this warp's 32 rows (lane quarter warp % 4), columns of this half of the block
-      tmem_st32(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + kTmemA + 64u * s + 32u * h, hv);
+      const uint32_t ta = tmem + kTmemA + 64u * s, sb = bstage(s);
+#pragma unroll
+      for (int ks = 0; ks < kTileK / 16; ++ks) {  // K = 16: 8 tensor-memory columns of A
+        const uint32_t slab = ks >> 2, koff = (ks & 3) * 32;
+        const int i = kb * (kTileK / 16) + ks;    // MMA number; accumulator i % nacc
+        mma_f16_ts_warp(tmem + static_cast<uint32_t>((i & (a.nacc - 1)) * a.tile_m), ta + 8u * ks,
+                        sw128_desc(sb + slab * slab_b + koff), idesc, i >= a.nacc ? 1u : 0u);
+      }
+      mma_commit_warp(empty + 8 * s);  // the stage is free once these MMAs are done
+    }
+    mma_commit_warp(accum);  // the accumulator is complete once every MMA is done
+  } else if (warp == 2) {
+    // ---------------- packed weights: 128 rows x 4 blocks per copy (rows past N read 0)
+    if (lane == 0) {
+      prefetch_tmap(&tm_w);
+      int issued = 0;
+      for (int c = 0; c < nchunks; ++c) {
+        const int r = c % kRawStages;
+        const uint32_t use = static_cast<uint32_t>(c / kRawStages);
+        if (!mbar_wait(emptyR + 8 * r, (use & 1) ^ 1, a.fault, kFaultW)) break;
+        ++issued;
+        mbar_arrive_expect_tx(fullR + 8 * r, kRawStageBytes);
+        tma_load_2d(rawring + r * kRawStageBytes, &tm_w,
+                    static_cast<int32_t>((kb0 / kChunkBlocks + c) * kChunkRowBytes),
+                    static_cast<int32_t>(n0), fullR + 8 * r);
+      }
+      for (int c = issued - kRawStages > 0 ? issued - kRawStages : 0; c < issued; ++c)
+        mbar_wait(fullR + 8 * (c % kRawStages), static_cast<uint32_t>(c / kRawStages) & 1,
+                  a.fault, kFaultW, /*give_up_after_fault=*/false);
+    }
+  } else if (warp >= 4) {
+    // ---------------- decode: thread d owns row d % 128, quarter r = d / 128 of each block
+    const int d = tid - 128;
+    const int row = d & (kTileN - 1), r4 = d >> 7;
+    const uint32_t base_e = tab | (static_cast<uint32_t>(lane & 15) << 3), base_o = base_e + 128u;
+    const uint32_t tlane = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + kTmemA + 16u * r4;
+    bool ok = true;
+    int kb = 0;  // blocks whose store has been issued
+    uint32_t hv[16];
+    // the previous block's store has landed: hand its stage to the MMA
+    auto publish_prev = [&]() {
       tmem_st_wait();
       tc_fence_before_sync();
-      mbar_arrive(fullA + 8 * s);
+      mbar_arrive(fullA + 8 * ((kb - 1) % kStagesTC));
+    };
+    // store block kb once the MMA has released its stage; completes during the next decode
+    auto store = [&]() {
+      const int s = kb % kStagesTC;
+      if (ok) ok = mbar_wait(empty + 8 * s, (static_cast<uint32_t>(kb / kStagesTC) & 1) ^ 1, a.fault,
+                             kFaultDecode);
+      __syncwarp();  // tcgen05.st is warp-collective
+      tc_fence_after_sync();
+      tmem_st16(tlane + 64u * s, hv);
+      ++kb;
+    };
+#pragma unroll 1
+    for (int c = 0; c < nchunks; ++c) {
+      const int r = c % kRawStages;
+      if (ok) ok = mbar_wait(fullR + 8 * r, static_cast<uint32_t>(c / kRawStages) & 1, a.fault, kFaultDecode);
+      uint4 raw[7];
+      const uint32_t src = rawring + r * kRawStageBytes + static_cast<uint32_t>(row) * kChunkRowBytes;
+#pragma unroll
+      for (int q = 0; q < 7; ++q) raw[q] = lds_u128(src + 16u * q);
+      mbar_arrive(emptyR + 8 * r);
+      decode_quarter<0>(raw, r4, base_e, base_o, hv);
+      if (kb > 0) publish_prev();
+      store();
+      if (kb < nkb) {
+        decode_quarter<1>(raw, r4, base_e, base_o, hv);
+        publish_prev();
+        store();
+      }
+      if (kb < nkb) {
+        decode_quarter<2>(raw, r4, base_e, base_o, hv);
+        publish_prev();
+        store();
+      }
+      if (kb < nkb) {
+        decode_quarter<3>(raw, r4, base_e, base_o, hv);
+        publish_prev();
+        store();
+      }
     }
-    cp_async_wait<0>();
+    if (kb > 0) publish_prev();
 
     // ---------------- epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (its rows);
-    // the two warp groups take alternate 16-column chunks
+    // the four warp groups take turns at 16-column chunks
     if (ok) ok = mbar_wait(accum, 0, a.fault, kFaultEpilogue);
     tc_fence_after_sync();
     const int q = warp & 3, grp = (warp - 4) >> 2;
     const int64_t ne = n0 + 32 * q + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
-    for (int c0 = 16 * grp; c0 < a.tile_m; c0 += 32) {
+    // every accumulator received at least one MMA: K >= 128 gives 8 per block
+    const int nacc_used = a.nacc < 8 * nkb ? a.nacc : 8 * nkb;
+    for (int c0 = 16 * grp; c0 < a.tile_m; c0 += 64) {
       uint32_t v[16];
       tmem_ld16(lane_base + static_cast<uint32_t>(c0), v);
       tmem_ld_wait();
+      for (int j = 1; j < nacc_used; ++j) {  // accumulators summed in order
+        uint32_t u[16];
+        tmem_ld16(lane_base + static_cast<uint32_t>(j * a.tile_m + c0), u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(u[i]));
+      }
       if (!ok || ne >= a.N) continue;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -402,11 +483,13 @@ TcPlan plan_for(const lbq_weights* w, int64_t M) {
   p.tile_m = M >= kMaxTileM ? kMaxTileM : static_cast<int>((M + 15) / 16 * 16);
   const int64_t tiles = ((w->N + kTileN - 1) / kTileN) * ((M + p.tile_m - 1) / p.tile_m);
   const int nkb = static_cast<int>(w->K / kTileK);
+  const int nchunks = (nkb + kChunkBlocks - 1) / kChunkBlocks;
   int splits = 1;
   if (tiles < sm_count()) splits = static_cast<int>(sm_count() / tiles);
-  if (splits > nkb) splits = nkb;
+  if (splits > nchunks) splits = nchunks;
   if (splits < 1) splits = 1;
-  p.kb_per_split = (nkb + splits - 1) / splits;
+  // whole chunks per split: a weight copy never straddles two splits
+  p.kb_per_split = (nchunks + splits - 1) / splits * kChunkBlocks;
   p.splits = (nkb + p.kb_per_split - 1) / p.kb_per_split;
   return p;
 }
@@ -456,8 +539,6 @@ cudaError_t lbq_launch_gemm_tc(const lbq_weights* w, const uint16_t* X, int64_t 
   if (e != cudaSuccess) return e;
 
   TcArgs a;
-  a.codes = static_cast<const uint8_t*>(w->codes);
-  a.cstride = w->code_stride;
   a.K = w->K;
   a.N = w->N;
   a.M = M;
@@ -465,12 +546,13 @@ cudaError_t lbq_launch_gemm_tc(const lbq_weights* w, const uint16_t* X, int64_t 
   a.Y = Y;
   const TcPlan plan = plan_for(w, M);
   a.tile_m = plan.tile_m;
+  a.nacc = 1;
+  while (a.nacc < 8 && 2 * a.nacc * a.tile_m <= static_cast<int>(kAccCols)) a.nacc *= 2;
   a.kb_per_split = plan.kb_per_split;
   a.part = plan.splits > 1
                ? reinterpret_cast<float*>(reinterpret_cast<char*>(xexp) +
                                           align_up(static_cast<size_t>(M) * sizeof(int), 256))
                : nullptr;
-  a.tmem_cols = a.tile_m <= 32 ? 32u : (a.tile_m <= 64 ? 64u : 128u);
   a.fault = lbq_fault_word();
   if (!a.fault) return cudaErrorInvalidDevicePointer;
 
@@ -485,9 +567,19 @@ cudaError_t lbq_launch_gemm_tc(const lbq_weights* w, const uint16_t* X, int64_t 
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  // packed weights as bytes [N][code_stride]: 112-byte x 128-row boxes, rows past N
+  // and bytes past the stride read as zero
+  CUtensorMap tw;
+  const cuuint64_t wdims[2] = {static_cast<cuuint64_t>(w->code_stride), static_cast<cuuint64_t>(w->N)};
+  const cuuint64_t wstrides[1] = {static_cast<cuuint64_t>(w->code_stride)};
+  const cuuint32_t wbox[2] = {kChunkRowBytes, static_cast<cuuint32_t>(kTileN)};
+  if (fn(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(w->codes), wdims, wstrides, wbox, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   dim3 grid(static_cast<unsigned>((w->N + kTileN - 1) / kTileN),
             static_cast<unsigned>((M + a.tile_m - 1) / a.tile_m), static_cast<unsigned>(plan.splits));
-  gemm_tern_tc_kernel<<<grid, kThreadsTC, kSmemTC, s>>>(tm, a);
+  gemm_tern_tc_kernel<<<grid, kThreadsTC, kSmemTC, s>>>(tm, tw, a);
   e = cudaGetLastError();
   if (e != cudaSuccess || plan.splits == 1) return e;
   const int64_t MN = M * w->N;
