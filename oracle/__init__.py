@@ -151,3 +151,35 @@ def gemm(fmt: int, codes: np.ndarray, scales, K: int, X_bf16_bits: np.ndarray, D
     _check(lib().orc_gemm(fmt, _ptr(codes), _ptr(sc), K, N, _ptr(X2), M, _ptr(Dp), _ptr(Y),
                           _ptr(B), int(nthreads)), "gemm")
     return Y, B
+
+
+def group4(a: np.ndarray) -> np.ndarray:
+    """Device order of a per-row array: rows interleaved in groups of four.
+
+    This is the library's own storage order (the pages fix no byte layout). Rows
+    are padded with zero rows to a multiple of four; in group g (rows 4g .. 4g+3),
+    element e of row 4g+q goes to position e*4 + q, where an "element" is one
+    32-bit word of a code row (uint8 input, row length a multiple of 4 bytes) or
+    one fp16 scale (uint16 input). Returns [ceil(N/4)][4 * row length] of the
+    input dtype.
+    """
+    a = np.ascontiguousarray(a)
+    N, R = a.shape
+    G = (N + 3) // 4
+    pad = np.zeros((4 * G, R), dtype=a.dtype)
+    pad[:N] = a
+    if a.dtype == np.uint8:
+        assert R % 4 == 0, "code rows hold whole 32-bit words"
+        return pad.reshape(G, 4, R // 4, 4).transpose(0, 2, 1, 3).reshape(G, 4 * R)
+    assert a.dtype == np.uint16, "codes (uint8) or fp16 scale bits (uint16)"
+    return pad.reshape(G, 4, R).transpose(0, 2, 1).reshape(G, 4 * R)
+
+
+def ungroup4(g: np.ndarray, N: int) -> np.ndarray:
+    """Inverse of group4: [ceil(N/4)][4 R] device order -> [N][R] rows."""
+    g = np.ascontiguousarray(g)
+    G, R4 = g.shape
+    R = R4 // 4
+    if g.dtype == np.uint8:
+        return g.reshape(G, R // 4, 4, 4).transpose(0, 2, 1, 3).reshape(4 * G, R)[:N]
+    return g.reshape(G, R, 4).transpose(0, 2, 1).reshape(4 * G, R)[:N]

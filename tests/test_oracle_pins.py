@@ -377,3 +377,44 @@ def test_gemm_threads_do_not_change_results(orc):
     Y1, B1 = orc.gemm(TERN5, codes, None, K, _bits(X), nthreads=1)
     Y4, B4 = orc.gemm(TERN5, codes, None, K, _bits(X), nthreads=4)
     assert np.array_equal(Y1, Y4) and np.array_equal(B1, B4)
+
+
+# ------------------------------------------------------------------ device row order
+
+def _read_group4_golden():
+    blocks, cur = {}, None
+    for line in open(os.path.join(GOLDEN, "group4_example.txt")):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        if line.startswith(("codes", "scales")):
+            cur = blocks.setdefault(line, [])
+            continue
+        cur.extend(int(v) for v in line.split())
+    return blocks
+
+
+def test_group4_worked_example(orc):
+    gold = _read_group4_golden()
+    codes = np.arange(80, dtype=np.uint8).reshape(5, 16)
+    g = orc.group4(codes)
+    assert g.shape == (2, 64)
+    assert g[0].tolist() == gold["codes group 0"]
+    assert g[1].tolist() == gold["codes group 1"]
+    sc = (np.arange(3)[:, None] * 10 + np.arange(2)[None, :] + 1).astype(np.uint16)
+    assert orc.group4(sc)[0].tolist() == gold["scales group 0"]
+
+
+@pytest.mark.parametrize("N", [1, 3, 4, 9])
+def test_group4_is_a_padded_permutation(orc, N):
+    rng = np.random.default_rng(N)
+    codes = rng.integers(0, 243, size=(N, 32), dtype=np.uint8)
+    g = orc.group4(codes)
+    assert g.shape == ((N + 3) // 4, 128)
+    # same multiset of bytes plus the zero padding rows, and exactly invertible
+    assert np.array_equal(np.sort(g.ravel()),
+                          np.sort(np.concatenate([codes.ravel(),
+                                                  np.zeros(g.size - codes.size, np.uint8)])))
+    assert np.array_equal(orc.ungroup4(g, N), codes)
+    sc = rng.integers(0, 1 << 16, size=(N, 5), dtype=np.uint16)
+    assert np.array_equal(orc.ungroup4(orc.group4(sc), N), sc)
