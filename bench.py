@@ -363,12 +363,15 @@ def sampled_parity(L, synth, prods, fmt, M, D, ws, args, dev, torch):
         torch.cuda.synchronize()
         W = synth.weights(p["N"], p["K"], synth.seed_of(args.seed * 1000, p["layer"], p["mi"]),
                           device=dev)
-        rows = np.sort(rng.choice(p["N"], size=min(48, p["N"]), replace=False))
+        # whole groups of four rows (the library's storage order), 12 of them
+        groups = np.sort(rng.choice(p["N"] // 4, size=min(12, p["N"] // 4), replace=False))
+        rows = (4 * groups[:, None] + np.arange(4)[None, :]).ravel()
         Wr = W[torch.from_numpy(rows).to(dev)].cpu().numpy()
         del W
         codes, scales = oracle.pack(fmt, Wr)
-        got_codes = p["pw"].codes[torch.from_numpy(rows).to(dev)].cpu().numpy()
-        assert np.array_equal(codes, got_codes), "timed weights differ from the oracle's packing"
+        got_codes = p["pw"].codes[torch.from_numpy(groups).to(dev)].cpu().numpy()
+        assert np.array_equal(oracle.group4(codes), got_codes), \
+            "timed weights differ from the oracle's packing"
         Xs = p["X"][: min(M, 8)]
         Do = oracle.rht_signs(args.seed * 31 + p["K"], p["K"]) if fmt == 3 else None
         Y, B = oracle.gemm(fmt, codes, scales, p["K"], synth.bf16_bits(Xs), Do,

@@ -80,8 +80,9 @@ lbq_status lbq_packed_layout(int32_t fmt, int64_t K, int64_t N, int64_t* code_st
   if (N < 1 || !lbq::layout_of(fmt, K, &L)) return LBQ_ERR_SHAPE;
   if (code_stride) *code_stride = L.code_stride;
   if (scale_stride) *scale_stride = L.scale_stride;
-  if (code_bytes) *code_bytes = static_cast<size_t>(N) * static_cast<size_t>(L.code_stride);
-  if (scale_bytes) *scale_bytes = static_cast<size_t>(N) * static_cast<size_t>(L.scale_stride) * 2;
+  const size_t rows = static_cast<size_t>(lbq::g4_rows(N));  // padded to whole groups of four
+  if (code_bytes) *code_bytes = rows * static_cast<size_t>(L.code_stride);
+  if (scale_bytes) *scale_bytes = rows * static_cast<size_t>(L.scale_stride) * 2;
   return LBQ_OK;
 }
 

@@ -13,18 +13,23 @@ namespace {
 using namespace lbq;
 
 template <int FMT>
-__device__ __forceinline__ float row_dot(const uint8_t* __restrict__ crow,
-                                         const uint16_t* __restrict__ srow, int64_t K,
+__device__ __forceinline__ float row_dot(const uint8_t* __restrict__ codes, int64_t cstride,
+                                         const uint16_t* __restrict__ scales, int64_t sstride,
+                                         int64_t n, int64_t K,
                                          const uint16_t* __restrict__ xb16,
                                          const float* __restrict__ xf32) {
   const int lane = threadIdx.x & 31;
   float acc = 0.0f;
+  // word i and scale b of row n in the group-of-four storage order
+  auto word = [&](int64_t i) -> uint32_t {
+    return *reinterpret_cast<const uint32_t*>(codes + g4_word_byte(n, i, cstride));
+  };
+  auto scale = [&](int64_t b) -> float { return f16_bits_to_f32(scales[g4_scale_elem(n, b, sstride)]); };
   if (FMT == LBQ_TERN5) {
-    const uint32_t* row = reinterpret_cast<const uint32_t*>(crow);
     for (int64_t b = lane; b < K / kTernBlock; b += 32) {
       uint32_t w[7];
 #pragma unroll
-      for (int q = 0; q < 7; ++q) w[q] = row[b * 7 + q];
+      for (int q = 0; q < 7; ++q) w[q] = word(b * 7 + q);
       const float s = f16_bits_to_f32(static_cast<uint16_t>(w[6] >> 16));
       float part = 0.0f;
 #pragma unroll
@@ -41,33 +46,31 @@ __device__ __forceinline__ float row_dot(const uint8_t* __restrict__ crow,
       acc += s * part;
     }
   } else if (FMT == LBQ_SIGN1) {
-    const uint32_t* row = reinterpret_cast<const uint32_t*>(crow);
     for (int64_t b = lane; b < K / kSignBlock; b += 32) {
       float part = 0.0f;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const uint32_t bits = row[b * 4 + q];
+        const uint32_t bits = word(b * 4 + q);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float xv = bf16_bits_to_f32(xb16[b * kSignBlock + 32 * q + i]);
           part += ((bits >> i) & 1u) ? xv : -xv;
         }
       }
-      acc += f16_bits_to_f32(srow[b]) * part;
+      acc += scale(b) * part;
     }
   } else {
-    const uint32_t* row = reinterpret_cast<const uint32_t*>(crow);
     for (int64_t b = lane; b < K / kQ2Block; b += 32) {
       float part = 0.0f;
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
-        const uint32_t bits = row[b * 2 + q];
+        const uint32_t bits = word(b * 2 + q);
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           part += (static_cast<float>((bits >> (2 * i)) & 3u) - 1.5f) *
                   xf32[b * kQ2Block + 16 * q + i];
       }
-      acc += f16_bits_to_f32(srow[b]) * part;
+      acc += scale(b) * part;
     }
   }
   return warp_sum(acc);
@@ -85,10 +88,9 @@ __global__ void __launch_bounds__(256) gemm_rowwarp(const uint8_t* __restrict__ 
   if (n >= N) return;
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * m_per_cta;
   const int64_t m1 = m0 + m_per_cta < M ? m0 + m_per_cta : M;
-  const uint8_t* crow = codes + n * cstride;
-  const uint16_t* srow = scales ? scales + n * sstride : nullptr;
   for (int64_t m = m0; m < m1; ++m) {
-    const float v = row_dot<FMT>(crow, srow, K, X + m * K, Xr ? Xr + m * K : nullptr);
+    const float v = row_dot<FMT>(codes, cstride, scales, sstride, n, K, X + m * K,
+                                 Xr ? Xr + m * K : nullptr);
     if ((threadIdx.x & 31) == 0) Y[m * N + n] = f32_to_bf16_bits(v);
   }
 }

@@ -47,9 +47,15 @@ constexpr int kMaxTileM = 128;  // tokens per tile (MMA N)
 constexpr int kStagesTC = 4;
 constexpr int kDecoders = 4 * kTileN;  // four threads per weight row, a quarter block each
 constexpr int kThreadsTC = 128 + kDecoders;
-constexpr int kChunkBlocks = 4;        // packed blocks per weight copy: 112 bytes, a multiple of 16
-constexpr uint32_t kChunkRowBytes = kChunkBlocks * kTernBlockBytes;
-constexpr uint32_t kRawStageBytes = kChunkRowBytes * kTileN;
+constexpr int kChunkBlocks = 4;        // packed blocks per weight copy: 28 words of each row
+constexpr uint32_t kChunkWords = kChunkBlocks * kTernBlockBytes / 4;
+// The rows arrive in groups of four (word w of four rows in 16 consecutive bytes).
+// A copy takes 32 groups x 116 words: the chunk's 112 words of each group plus the
+// next chunk's first four, so that a group's row in shared memory is 464 bytes (29
+// 16-byte bank groups, an odd number): the 32 rows a warp decodes then read their
+// words from 32 different banks.
+constexpr uint32_t kGroupWords = 4 * kChunkWords + 4;
+constexpr uint32_t kRawStageBytes = kGroupWords * 4 * (kTileN / 4);
 constexpr int kRawStages = 2;
 constexpr uint32_t kStageB = 2 * kMaxTileM * 128;  // two 64-k slabs of activations
 // Tensor memory (512 columns): nacc fp32 accumulators of tile_m columns each in
@@ -156,6 +162,11 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
   return d;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
 }
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   uint2 v;
@@ -325,8 +336,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         ++issued;
         mbar_arrive_expect_tx(fullR + 8 * r, kRawStageBytes);
         tma_load_2d(rawring + r * kRawStageBytes, &tm_w,
-                    static_cast<int32_t>((kb0 / kChunkBlocks + c) * kChunkRowBytes),
-                    static_cast<int32_t>(n0), fullR + 8 * r);
+                    static_cast<int32_t>((kb0 / kChunkBlocks + c) * 4 * kChunkWords),
+                    static_cast<int32_t>(n0 / 4), fullR + 8 * r);
       }
       for (int c = issued - kRawStages > 0 ? issued - kRawStages : 0; c < issued; ++c)
         mbar_wait(fullR + 8 * (c % kRawStages), static_cast<uint32_t>(c / kRawStages) & 1,
@@ -362,9 +373,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const int r = c % kRawStages;
       if (ok) ok = mbar_wait(fullR + 8 * r, static_cast<uint32_t>(c / kRawStages) & 1, a.fault, kFaultDecode);
       uint4 raw[7];
-      const uint32_t src = rawring + r * kRawStageBytes + static_cast<uint32_t>(row) * kChunkRowBytes;
+      // word w of this row: group row >> 2, element 4 w + (row & 3) of the group
+      const uint32_t src = rawring + r * kRawStageBytes +
+                           4u * (static_cast<uint32_t>(row >> 2) * kGroupWords + (row & 3));
 #pragma unroll
-      for (int q = 0; q < 7; ++q) raw[q] = lds_u128(src + 16u * q);
+      for (int q = 0; q < 7; ++q)
+        raw[q] = make_uint4(lds32(src + 64u * q), lds32(src + 64u * q + 16u),
+                            lds32(src + 64u * q + 32u), lds32(src + 64u * q + 48u));
       mbar_arrive(emptyR + 8 * r);
       decode_quarter<0>(raw, r4, base_e, base_o, hv);
       if (kb > 0) publish_prev();
@@ -567,13 +582,15 @@ cudaError_t lbq_launch_gemm_tc(const lbq_weights* w, const uint16_t* X, int64_t 
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  // packed weights as bytes [N][code_stride]: 112-byte x 128-row boxes, rows past N
-  // and bytes past the stride read as zero
+  // packed weights as 32-bit words, one row of the map per group of four rows
+  // (code_stride words); boxes of 116 words x 32 groups; groups past the end and
+  // words past the row read as zero
   CUtensorMap tw;
-  const cuuint64_t wdims[2] = {static_cast<cuuint64_t>(w->code_stride), static_cast<cuuint64_t>(w->N)};
-  const cuuint64_t wstrides[1] = {static_cast<cuuint64_t>(w->code_stride)};
-  const cuuint32_t wbox[2] = {kChunkRowBytes, static_cast<cuuint32_t>(kTileN)};
-  if (fn(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(w->codes), wdims, wstrides, wbox, estr,
+  const cuuint64_t wdims[2] = {static_cast<cuuint64_t>(w->code_stride),
+                               static_cast<cuuint64_t>((w->N + 3) / 4)};
+  const cuuint64_t wstrides[1] = {static_cast<cuuint64_t>(w->code_stride) * 4};
+  const cuuint32_t wbox[2] = {kGroupWords, static_cast<cuuint32_t>(kTileN / 4)};
+  if (fn(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(w->codes), wdims, wstrides, wbox, estr,
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;

@@ -7,32 +7,34 @@
 // input x' = H D x / sqrt(512) of the feinterview.poetries.top "27B in 12 GB"
 // article, computed here in shared memory, never in global memory.
 //
-// Design (HBM-bound: the decode must cost about one instruction per weight):
-//  * Lookup of partial sums. A CTA owns one K-slice at a time (ternary: 4 blocks,
-//    512 weights, 28 words of a row; 1-bit: 1024 weights, 32 words; 2-bit: 512
+// Design (HBM-bound: about one issued instruction per weight is all there is):
+//  * Lookup of partial sums. A CTA owns one K-slice (ternary: 4 blocks, 512
+//    weights, 28 words of a row; 1-bit: 1024 weights, 32 words; 2-bit: 512
 //    weights, 32 words) and builds in shared memory, for every byte position of the
 //    slice, the partial dot product of that byte's codes with the slice of x, for
-//    all 256 byte values. A byte then costs one PRMT (which forms the table address
-//    directly), one LDS and one add. The table is laid out [value][lane], lane l
-//    always reads word l of a row, so table reads are bank-conflict free.
-//  * Warp specialisation. One producer lane streams 32-row x slice tiles of codes
-//    (and, for the 1-bit and 2-bit formats, of scales) with 2D TMA into a ring of
-//    shared-memory stages guarded by mbarriers; ragged edges arrive zero-filled.
-//    Sixteen consumer warps each take one 32-row unit at a time. At step g lane l
-//    works on row g ^ l of the unit (rows visited in Gray-code order, so the row
-//    address moves by one signed power of two per step); every read stays
-//    conflict-free and a select-free butterfly then leaves row l's sum in lane l.
-//  * Split-K. Slices are spread over CTAs; each unit's 32 sums go to the workspace,
-//    and a small second kernel (launched with programmatic dependent launch, so it
-//    starts while the first is finishing) adds each row's slice sums in slice order
-//    and writes bf16 y: results are deterministic. (Folding that sum into the main
-//    kernel, with the last of a row group's CTAs doing it, measured slightly slower.)
-//    A matrix of one slice writes y directly.
-//  * Grid of floor(SMs / slices) CTAs per slice, one CTA per SM, each with an equal
-//    share of its slice's 32-row chunks, so that no CTA builds a second table.
-//    Programmatic dependent launch:
-//    the producer streams weights before the previous kernel in the stream has
-//    finished; consumers wait for it before touching x, y or the workspace.
+//    all 256 byte values (128 KB). A byte then costs one PRMT (which forms the
+//    table address from the byte and the lane), one LDS and one add. Lane l always
+//    handles the same word position of a row, and the table is laid out
+//    [value][lane], so table reads never collide on a bank.
+//  * Streaming. The packed rows are stored in groups of four (word w of four rows
+//    in 16 consecutive bytes), so one coalesced 16-byte load per lane brings a
+//    lane its word of four rows: a warp load covers 448 (ternary) or 512 bytes.
+//    Loads go straight to registers, three 16-row units in flight per warp; no
+//    shared-memory staging, whose extra write and read would cost shared-memory
+//    bandwidth, the kernel's second bound.
+//  * Reduction. Each lane holds one word's partial sum for each of 16 rows; a
+//    transpose-reduce butterfly (15 shuffles) leaves row l's slice sum in lane l.
+//  * Scales. Ternary scales live in word 6 of each 28-byte block: lanes are mapped
+//    so that block b is lanes 8b .. 8b+6, and lane 8b+6 hands each pair of rows'
+//    scales to its block's lanes with one shuffle. 1-bit and 2-bit scales come
+//    with one 8-byte load per lane per four rows (group-of-four scale order).
+//  * Split-K. Slices are spread over CTAs; slice sums go to the workspace and a
+//    small second kernel (programmatic dependent launch) adds each row's slice
+//    sums in slice order and writes bf16 y: results are deterministic.
+//  * Programmatic dependent launch: before waiting for the previous kernel, each
+//    warp asks L2 to prefetch its first units of weights (a hint only: the loads
+//    that feed the arithmetic are issued after the wait, so weights written by the
+//    previous kernel are always read correctly).
 #include <cudaTypedefs.h>
 
 #include "rht.cuh"
@@ -42,105 +44,49 @@ namespace {
 
 using namespace lbq;
 
-constexpr int kMaxConsumers = 16;               // consumer warps (per format, see Traits)
-constexpr int kMaxThreads = 32 * (kMaxConsumers + 1);  // + one producer warp
-constexpr int kRows = 32;                       // rows per unit
-constexpr int kMaxStages = 32;
-constexpr uint32_t kPage = 65536;               // table page: 256 values x 256 bytes
-constexpr uint32_t kTailBytes = 4096 + 2 * kMaxStages * 8;  // x slice + mbarriers
-// Shared memory layout. The table must start on a 64 KB boundary of the shared
-// window (its page addressing keeps the base in the upper half of the PRMT
-// operand), and the dynamic allocation does not start on one (the first 1 KB of
-// the window is reserved). So the whole opt-in maximum is requested: the table
-// sits at the first 64 KB boundary, the stages fill the space below it and
-// continue above it, followed by the x slice and the mbarriers. There are more
-// stages than consumer warps, so each warp's next unit streams in while it works
-// on the current one. The request is sized for a window starting at 0 or 1 KB, and
-// leaves room on the SM for a CTA of the small split-K sum kernel.
-constexpr uint32_t smem_bytes(uint32_t stage, uint32_t stages) {
-  // window starting at 1 KB: stages below the table, the rest above it
-  const uint32_t below = (kPage - 1024) / stage < stages ? (kPage - 1024) / stage : stages;
-  const uint32_t at_1k = (kPage - 1024) + 2 * kPage + (stages - below) * stage + kTailBytes;
-  // window starting at 0: everything above the table
-  const uint32_t at_0 = 2 * kPage + stages * stage + kTailBytes;
-  return at_1k > at_0 ? at_1k : at_0;
-}
-constexpr unsigned kFaultProducer = 1, kFaultConsumer = 2, kFaultLayout = 3;
+constexpr int kWarps = 16;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kRows = 16;           // rows per unit (four groups of four)
+constexpr int kAhead = 3;           // units in flight per warp
+constexpr uint32_t kPage = 65536;   // table page: 256 values x 256 bytes
+// Shared memory: the 128 KB table at the first 64 KB boundary of the window (its
+// page addressing keeps the base in the upper half of the PRMT operand), the x
+// slice below it. The dynamic window starts 1 KB into shared memory on sm_100, so
+// [1 KB, 64 KB) holds the x slice; a window starting at 0 puts x above the table.
+constexpr uint32_t kXBytes = 4096;  // up to 1024 fp32
+constexpr uint32_t kSmem = (kPage - 1024) + 2 * kPage + kXBytes;
+constexpr unsigned kFaultLayout = 3;
 
 template <int FMT>
 struct Traits;
 template <>
 struct Traits<LBQ_TERN5> {
-  static constexpr int kWeights = 512, kBlocks = 4, kPitch = 112;
-  static constexpr int kHi = 9;                 // value = lo + 27 * hi
-  static constexpr int kScaleBox = 0;           // scales live in the blocks
-  static constexpr uint32_t kStageCodes = 3584, kStageBytes = 3584;  // 32 x 112 bytes
-  static constexpr int kStages = 26;
-  static constexpr int kConsumers = 16;
-  static constexpr uint32_t kSmem = smem_bytes(kStageBytes, kStages);
+  static constexpr int kWeights = 512, kWords = 28, kBlocks = 4, kDigits = 5;
 };
 template <>
 struct Traits<LBQ_SIGN1> {
-  static constexpr int kWeights = 1024, kBlocks = 8, kPitch = 128;
-  static constexpr int kHi = 16;                // value = lo + 16 * hi
-  static constexpr int kScaleBox = 8;           // fp16 scales per row per slice
-  static constexpr uint32_t kStageCodes = 4096, kStageBytes = 4096 + 512;
-  static constexpr int kStages = 20;
-  static constexpr int kConsumers = 14;
-  static constexpr uint32_t kSmem = smem_bytes(kStageBytes, kStages);
+  static constexpr int kWeights = 1024, kWords = 32, kBlocks = 8, kDigits = 8;
 };
 template <>
 struct Traits<LBQ_Q2RHT> {
-  static constexpr int kWeights = 512, kBlocks = 16, kPitch = 128;
-  static constexpr int kHi = 16;
-  static constexpr int kScaleBox = 16;
-  static constexpr uint32_t kStageCodes = 4096, kStageBytes = 4096 + 1024;
-  static constexpr int kStages = 18;
-  static constexpr int kConsumers = 12;
-  static constexpr uint32_t kSmem = smem_bytes(kStageBytes, kStages);
+  static constexpr int kWeights = 512, kWords = 32, kBlocks = 16, kDigits = 4;
 };
 
-template <uint32_t kImm>
-__device__ __forceinline__ float lds_imm(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(kImm));
-  return v;
-}
-__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ uint16_t lds_u16(uint32_t addr) {
-  uint16_t v;
-  asm volatile("ld.shared.b16 %0, [%1];" : "=h"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ void sts_f2(uint32_t addr, float2 v) {
-  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(v.x), "f"(v.y) : "memory");
-}
-
-// Sum of the four table entries addressed by the bytes of w0 (.x) and of w1 (.y),
-// two rows at a time so the adds run packed. Slot i lives on page i/2 at column
-// offset (i%2)*128; `lanereg` = table base | lane*4.
-template <uint32_t kImm, uint32_t kSel>
-__device__ __forceinline__ float2 entry2(uint32_t w0, uint32_t w1, uint32_t lanereg) {
-  return make_float2(lds_imm<kImm>(__byte_perm(w0, lanereg, kSel)),
-                     lds_imm<kImm>(__byte_perm(w1, lanereg, kSel)));
-}
-__device__ __forceinline__ float2 lookup4x2(uint32_t w0, uint32_t w1, uint32_t lanereg) {
-  const float2 e0 = entry2<0, 0x7604>(w0, w1, lanereg);
-  const float2 e1 = entry2<128, 0x7614>(w0, w1, lanereg);
-  const float2 e2 = entry2<kPage, 0x7624>(w0, w1, lanereg);
-  const float2 e3 = entry2<kPage + 128, 0x7634>(w0, w1, lanereg);
-  return __fadd2_rn(__fadd2_rn(e0, e1), __fadd2_rn(e2, e3));
-}
-
-// Weight index (within the slice) of digit e of the byte in table column (slot, w),
-// or -1 if that digit carries no weight (scale bytes, padding, idle lanes).
+// Word of the slice that lane l handles (ternary: block l/8, word l%8 of it; lanes
+// 7, 15, 23, 31 have none), or -1; nb = blocks present in this slice.
 template <int FMT>
-__device__ __forceinline__ int digit_weight(int slot, int w, int e, int nw) {
-  if (w >= nw) return -1;
+__device__ __forceinline__ int lane_word(int l, int nb) {
+  if (FMT == LBQ_TERN5) return ((l & 7) < 7 && (l >> 3) < nb) ? 7 * (l >> 3) + (l & 7) : -1;
+  if (FMT == LBQ_SIGN1) return l < 4 * nb ? l : -1;
+  return l;
+}
+
+// Weight index (within the slice) of digit e of byte `slot` of lane l's word, or -1
+// if that digit carries no weight (scale bytes, byte-25 padding digits, no word).
+template <int FMT>
+__device__ __forceinline__ int digit_weight(int slot, int l, int e, int nb) {
+  const int w = lane_word<FMT>(l, nb);
+  if (w < 0) return -1;
   if (FMT == LBQ_TERN5) {
     const int bb = w / 7, c = 4 * (w % 7) + slot;  // byte within the 28-byte block
     if (c >= kTernCodeBytes) return -1;            // the block's fp16 scale
@@ -153,52 +99,83 @@ __device__ __forceinline__ int digit_weight(int slot, int w, int e, int nw) {
   }
 }
 
-// Address change when bit b of (g ^ lane) is set, for a row pitch p: +-p * 2^b.
-// Five named values (not an array) so that unrolled code keeps them in registers.
-struct Steps {
-  int32_t d0, d1, d2, d3, d4;
-  __device__ __forceinline__ Steps(int lane, int p)
-      : d0((lane & 1) ? -p : p),
-        d1((lane & 2) ? -2 * p : 2 * p),
-        d2((lane & 4) ? -4 * p : 4 * p),
-        d3((lane & 8) ? -8 * p : 8 * p),
-        d4((lane & 16) ? -16 * p : 16 * p) {}
-  __device__ __forceinline__ int32_t at(int b) const {
-    return b == 0 ? d0 : (b == 1 ? d1 : (b == 2 ? d2 : (b == 3 ? d3 : d4)));
-  }
-};
-
 template <int FMT>
 struct Args {
+  const uint8_t* codes;
+  const uint16_t* scales;
+  int64_t cstride;  // code bytes per row (a group of four rows is 4 * cstride)
+  int64_t sstride;  // scales per row
   int64_t K, N;
   const uint16_t* x;
   const int8_t* D;
   uint16_t* y;
-  float* part;    // [KS][N] slice sums (KS > 1)
-  int KS;         // number of slices
-  int G;          // CTAs per slice
-  int nblk;       // scale blocks per row
-  unsigned* fault;  // set when a bounded wait gives up
+  float* part;      // [KS][N] slice sums (KS > 1)
+  int KS;           // number of slices
+  int G;            // CTAs per slice
+  int nblk;         // scale blocks per row
+  unsigned* fault;  // set when the shared-memory layout check fails
 };
 
-// Builds the x slice and the lookup tables for slice j (consumer threads only).
-// Thread t owns table column pair t % 64 (two adjacent lanes of one byte slot) and
-// the values v = lo + R * hi for hi = t / 64, t / 64 + T/64, ...; everything that
-// does not depend on hi is computed once.
+__device__ __forceinline__ void sts_f2(uint32_t addr, float2 v) {
+  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(v.x), "f"(v.y) : "memory");
+}
+template <uint32_t kImm>
+__device__ __forceinline__ float lds_imm(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(kImm));
+  return v;
+}
+__device__ __forceinline__ uint4 ldg_stream16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint2 ldg_stream8(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.b32 {%0, %1}, [%2];"
+               : "=r"(v.x), "=r"(v.y)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ float2 h2_to_f2(uint32_t h2) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&h2));
+}
+
+// Table entries of one row word: the four bytes' partial sums added up.
+// Slot i lives on page i/2 at column offset (i%2)*128; `lanereg` = table base | lane*4.
+__device__ __forceinline__ float2 lookup_pair(uint32_t w0, uint32_t w1, uint32_t lanereg) {
+  const float2 e0 = make_float2(lds_imm<0>(__byte_perm(w0, lanereg, 0x7604)),
+                                lds_imm<0>(__byte_perm(w1, lanereg, 0x7604)));
+  const float2 e1 = make_float2(lds_imm<128>(__byte_perm(w0, lanereg, 0x7614)),
+                                lds_imm<128>(__byte_perm(w1, lanereg, 0x7614)));
+  const float2 e2 = make_float2(lds_imm<kPage>(__byte_perm(w0, lanereg, 0x7624)),
+                                lds_imm<kPage>(__byte_perm(w1, lanereg, 0x7624)));
+  const float2 e3 = make_float2(lds_imm<kPage + 128>(__byte_perm(w0, lanereg, 0x7634)),
+                                lds_imm<kPage + 128>(__byte_perm(w1, lanereg, 0x7634)));
+  return __fadd2_rn(__fadd2_rn(e0, e1), __fadd2_rn(e2, e3));
+}
+
+// Builds the x slice and the lookup table for slice j (all threads).
+// Thread t owns table column pair t % 64 (lanes 2c, 2c+1 of one byte slot) and the
+// values v = lo + R * hi for hi = t / 64, t / 64 + 8, ...; everything that does not
+// depend on hi is computed once.
 template <int FMT>
 __device__ __forceinline__ void build_slice(const Args<FMT>& a, int32_t j, uint32_t tbase,
-                                            float* xs, int ctid) {
+                                            float* xs, int tid) {
   using T = Traits<FMT>;
-  constexpr int kCT = 32 * T::kConsumers;
   const int blk0 = j * T::kBlocks;
-  const int nb_here = a.nblk - blk0 < T::kBlocks ? a.nblk - blk0 : T::kBlocks;
-  const int nw = FMT == LBQ_TERN5 ? 7 * nb_here : (FMT == LBQ_SIGN1 ? 4 * nb_here : 2 * nb_here);
-  const int nx = FMT == LBQ_Q2RHT ? nb_here * kQ2Block : nb_here * kTernBlock;
+  const int nb = a.nblk - blk0 < T::kBlocks ? a.nblk - blk0 : T::kBlocks;
+  const int nx = FMT == LBQ_Q2RHT ? nb * kQ2Block : nb * kTernBlock;
   const int64_t k0 = static_cast<int64_t>(j) * T::kWeights;
-  const int lane = ctid & 31;
+  const int lane = tid & 31;
 
   if (FMT == LBQ_Q2RHT) {
-    if (ctid < 32) {
+    if (tid < 32) {
       float v[16];
       rht512_warp_load(a.x + k0, a.D + k0, v);
       float4* d = reinterpret_cast<float4*>(xs + 16 * lane);
@@ -206,8 +183,8 @@ __device__ __forceinline__ void build_slice(const Args<FMT>& a, int32_t j, uint3
       for (int q = 0; q < 4; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
   } else {
-    // one 16-byte load of 8 activations per thread (x is 16-byte aligned, slices too)
-    for (int i = ctid; i < T::kWeights / 8; i += kCT) {
+    // one 16-byte load of 8 activations per thread (x and the slices are 16-byte aligned)
+    for (int i = tid; i < T::kWeights / 8; i += kThreads) {
       float f[8];
       if (8 * i < nx) {
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x + k0) + i);
@@ -226,28 +203,28 @@ __device__ __forceinline__ void build_slice(const Args<FMT>& a, int32_t j, uint3
       d[1] = make_float4(f[4], f[5], f[6], f[7]);
     }
   }
-  named_bar_sync(1, kCT);
+  __syncthreads();
 
-  const int cp = ctid & 63;
-  const int slot = cp >> 4, w0 = 2 * (cp & 15);
-  constexpr int kDigits = FMT == LBQ_TERN5 ? 5 : (FMT == LBQ_SIGN1 ? 8 : 4);
-  float2 xv[kDigits];
+  const int cp = tid & 63;
+  const int slot = cp >> 4, l0 = 2 * (cp & 15);
+  float2 xv[T::kDigits];
 #pragma unroll
-  for (int e = 0; e < kDigits; ++e) {
-    const int ka = digit_weight<FMT>(slot, w0, e, nw);
-    const int kb = digit_weight<FMT>(slot, w0 + 1, e, nw);
+  for (int e = 0; e < T::kDigits; ++e) {
+    const int ka = digit_weight<FMT>(slot, l0, e, nb);
+    const int kb = digit_weight<FMT>(slot, l0 + 1, e, nb);
     xv[e] = make_float2(ka >= 0 ? xs[ka] : 0.0f, kb >= 0 ? xs[kb] : 0.0f);
   }
-  const uint32_t col = tbase + (slot >> 1) * kPage + (slot & 1) * 128 + w0 * 4;
+  const uint32_t col = tbase + (slot >> 1) * kPage + (slot & 1) * 128 + l0 * 4;
+  constexpr int kStep = kThreads / 64;
   if (FMT == LBQ_TERN5) {
     // v = d0 + 3 d1 + 9 d2 + 27 (d3 + 3 d4); entry = sum_e (d_e - 1) x_e
     float2 ab[9];
 #pragma unroll
     for (int m = 0; m < 9; ++m) {
-      const float l0 = static_cast<float>(m % 3 - 1), l1 = static_cast<float>(m / 3 - 1);
-      ab[m] = __ffma2_rn(make_float2(l0, l0), xv[0], __fmul2_rn(make_float2(l1, l1), xv[1]));
+      const float l0f = static_cast<float>(m % 3 - 1), l1f = static_cast<float>(m / 3 - 1);
+      ab[m] = __ffma2_rn(make_float2(l0f, l0f), xv[0], __fmul2_rn(make_float2(l1f, l1f), xv[1]));
     }
-    for (int hi = ctid >> 6; hi < T::kHi; hi += kCT / 64) {
+    for (int hi = tid >> 6; hi < 9; hi += kStep) {
       const float l3 = static_cast<float>(hi % 3 - 1), l4 = static_cast<float>(hi / 3 - 1);
       const float2 q = __ffma2_rn(make_float2(l3, l3), xv[3], __fmul2_rn(make_float2(l4, l4), xv[4]));
 #pragma unroll
@@ -260,7 +237,7 @@ __device__ __forceinline__ void build_slice(const Args<FMT>& a, int32_t j, uint3
       }
     }
     // byte values 243..255 never occur: zero rows keep them harmless
-    for (int i = ctid; i < 13 * 64; i += kCT) {
+    for (int i = tid; i < 13 * 64; i += kThreads) {
       const int v = 243 + i / 64, c = i % 64;
       sts_f2(tbase + (c >> 5) * kPage + static_cast<uint32_t>(v) * 256u + (c & 31) * 8,
              make_float2(0.0f, 0.0f));
@@ -271,16 +248,16 @@ __device__ __forceinline__ void build_slice(const Args<FMT>& a, int32_t j, uint3
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       if (FMT == LBQ_SIGN1) {
-        const float l0 = (m & 1) ? 1.0f : -1.0f, l1 = (m & 2) ? 1.0f : -1.0f;
-        av[m] = __ffma2_rn(make_float2(l0, l0), xv[0], __fmul2_rn(make_float2(l1, l1), xv[1]));
-        bv[m] = __ffma2_rn(make_float2(l0, l0), xv[2], __fmul2_rn(make_float2(l1, l1), xv[3]));
+        const float s0 = (m & 1) ? 1.0f : -1.0f, s1 = (m & 2) ? 1.0f : -1.0f;
+        av[m] = __ffma2_rn(make_float2(s0, s0), xv[0], __fmul2_rn(make_float2(s1, s1), xv[1]));
+        bv[m] = __ffma2_rn(make_float2(s0, s0), xv[2], __fmul2_rn(make_float2(s1, s1), xv[3]));
       } else {
         const float l = static_cast<float>(m) - 1.5f;
         av[m] = __fmul2_rn(make_float2(l, l), xv[0]);
         bv[m] = __fmul2_rn(make_float2(l, l), xv[1]);
       }
     }
-    for (int hi = ctid >> 6; hi < T::kHi; hi += kCT / 64) {
+    for (int hi = tid >> 6; hi < 16; hi += kStep) {
       float2 q;
       if (FMT == LBQ_SIGN1) {
         q = make_float2(0.0f, 0.0f);
@@ -302,156 +279,122 @@ __device__ __forceinline__ void build_slice(const Args<FMT>& a, int32_t j, uint3
       }
     }
   }
-  named_bar_sync(1, kCT);
+  __syncthreads();
 }
 
 template <int FMT>
-__global__ void __launch_bounds__(kMaxThreads, 1)
-    gemv_lut_kernel(const __grid_constant__ CUtensorMap tm_codes,
-                    const __grid_constant__ CUtensorMap tm_scales, const Args<FMT> a) {
+__global__ void __launch_bounds__(kThreads, 1) gemv_lut_kernel(const Args<FMT> a) {
   using T = Traits<FMT>;
+  constexpr bool kSepScales = FMT != LBQ_TERN5;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_launch_dependents();
 
-  constexpr int kStages = T::kStages;
-  constexpr uint32_t kStageBytes = T::kStageBytes, kStageCodes = T::kStageCodes;
-  constexpr int kConsumers = T::kConsumers;
-  static_assert(kStages <= kMaxStages && kStages > kConsumers && kConsumers <= kMaxConsumers,
-                "stage ring");
   const uint32_t sbase = smem_u32(smem);
   const uint32_t tbase = (sbase + kPage - 1) & ~(kPage - 1);
-  const uint32_t n_low = (tbase - sbase) / kStageBytes < kStages ? (tbase - sbase) / kStageBytes
-                                                                 : kStages;
-  const uint32_t high = tbase + 2 * kPage;  // first byte above the table
-  const uint32_t tail = high + (kStages - n_low) * kStageBytes;
-  if (tail + kTailBytes > sbase + T::kSmem) {  // cannot happen with a 0 or 1 KB reserved prefix
-    if (tid == 0) atomicExch(a.fault, kFaultLayout);
+  const uint32_t xaddr = (tbase - sbase >= kXBytes) ? sbase : tbase + 2 * kPage;
+  if (tbase + 2 * kPage > sbase + kSmem || xaddr + kXBytes > sbase + kSmem) {
+    if (tid == 0) atomicExch(a.fault, kFaultLayout);  // cannot happen with a 0 or 1 KB prefix
     return;
   }
-  auto stage_addr = [&](int s) -> uint32_t {
-    return static_cast<uint32_t>(s) < n_low ? sbase + s * kStageBytes
-                                            : high + (s - n_low) * kStageBytes;
-  };
-  float* xs = reinterpret_cast<float*>(smem + (tail - sbase));
-  const uint32_t full0 = tail + 4096, empty0 = full0 + kStages * 8;
+  float* xs = reinterpret_cast<float*>(smem + (xaddr - sbase));
 
-  // This CTA: slice j, 32-row chunks [c_lo, c_hi) of it (a.G CTAs share a slice).
-  const int32_t NC = static_cast<int32_t>((a.N + kRows - 1) / kRows);
+  // This CTA: slice j, units [u_lo, u_hi) of kRows rows (a.G CTAs share a slice).
+  // 32-bit arithmetic: NU <= 2^15 and G <= the SM count.
+  const int32_t NU = static_cast<int32_t>((a.N + kRows - 1) / kRows);
+  const int32_t NG = static_cast<int32_t>((a.N + 3) / 4);  // groups of four rows present
   const int32_t j = static_cast<int32_t>(blockIdx.x) / a.G;
   const int32_t gs = static_cast<int32_t>(blockIdx.x) - j * a.G;
-  // (32-bit arithmetic: NC <= 16384 and G <= the SM count, so gs * NC fits; a 64-bit
-  // division here costs the kernel most of a microsecond)
-  const int32_t c_lo = static_cast<int32_t>(static_cast<uint32_t>(gs * NC) / static_cast<uint32_t>(a.G));
-  const int32_t c_hi =
-      static_cast<int32_t>(static_cast<uint32_t>((gs + 1) * NC) / static_cast<uint32_t>(a.G));
-  const int32_t n_units = c_hi - c_lo;
+  const int32_t u_lo = static_cast<int32_t>(static_cast<uint32_t>(gs * NU) / static_cast<uint32_t>(a.G));
+  const int32_t u_hi =
+      static_cast<int32_t>(static_cast<uint32_t>((gs + 1) * NU) / static_cast<uint32_t>(a.G));
+  const int32_t n_units = u_hi - u_lo;
 
-  if (tid < kStages) {  // one barrier pair per thread; each initialiser fences its own inits
-    mbar_init(full0 + 8 * tid, 1);
-    mbar_init(empty0 + 8 * tid, 1);
-    fence_mbar_init();
+  const int blk0 = j * T::kBlocks;
+  const int nb = a.nblk - blk0 < T::kBlocks ? a.nblk - blk0 : T::kBlocks;
+  const int wl = lane_word<FMT>(lane, nb);
+  const int64_t gstride = 4 * a.cstride;  // bytes per group of four rows
+  const uint8_t* slice = a.codes + static_cast<int64_t>(16) * j * T::kWords;
+  const uint8_t* cptr = slice + 16 * (wl < 0 ? 0 : wl);
+  // 1-bit / 2-bit: this lane's block scales of four rows are 8 bytes of the group
+  const int sblk = blk0 + (FMT == LBQ_SIGN1 ? (lane >> 2) : (lane >> 1));
+  const uint16_t* sptr = kSepScales ? a.scales + 4 * sblk : nullptr;
+  const int64_t sgstride = 4 * a.sstride;
+
+  // Ask L2 for this warp's first units (a hint; the real loads follow the wait).
+  if (lane < 4 * kAhead) {
+    const int32_t u = u_lo + warp + kWarps * (lane >> 2);
+    const int32_t g = 4 * u + (lane & 3);
+    const int64_t words_left = a.cstride / 4 - static_cast<int64_t>(j) * T::kWords;
+    const uint32_t bytes = 16u * static_cast<uint32_t>(words_left < T::kWords ? words_left : T::kWords);
+    if (u < u_hi && g < NG) prefetch_l2_bulk(slice + g * gstride, bytes);
   }
-  __syncthreads();
 
-  if (warp == kConsumers) {
-    // ---------------- producer: one lane streams tiles of codes (and scales)
-    if (lane == 0) {
-      prefetch_tmap(&tm_codes);
-      if (T::kScaleBox) prefetch_tmap(&tm_scales);
-      const uint32_t bytes = T::kPitch * kRows + T::kScaleBox * 2 * kRows;
-      int32_t issued = 0;
-      int s = 0;
-      uint32_t phase = 0;
-      for (int32_t c = c_lo; c < c_hi; ++c) {
-        if (!mbar_wait(empty0 + 8 * s, phase ^ 1, a.fault, kFaultProducer)) break;
-        ++issued;
-        mbar_arrive_expect_tx(full0 + 8 * s, bytes);
-        const uint32_t dst = stage_addr(s);
-        tma_load_2d(dst, &tm_codes, j * T::kPitch, c * kRows, full0 + 8 * s);
-        if (T::kScaleBox)
-          tma_load_2d(dst + kStageCodes, &tm_scales, j * T::kScaleBox, c * kRows, full0 + 8 * s);
-        if (++s == kStages) {
-          s = 0;
-          phase ^= 1;
-        }
-      }
-      // Before this lane exits, every copy it issued must have landed (normally the
-      // consumers have already seen them all; this matters only after a fault).
-      for (int s2 = 0; s2 < kStages && s2 < issued; ++s2) {
-        const int32_t k_last = s2 + (issued - 1 - s2) / kStages * kStages;
-        mbar_wait(full0 + 8 * s2, static_cast<uint32_t>(k_last / kStages) & 1, a.fault,
-                  kFaultProducer, /*give_up_after_fault=*/false);
-      }
+  uint4 buf[kAhead][4];
+  uint2 sbuf[kAhead][4];
+  auto load = [&](uint4 (&b)[4], uint2 (&sb)[4], int32_t u) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int32_t g = 4 * u + q;
+      const bool ok = u < u_hi && g < NG && wl >= 0;
+      b[q] = ok ? ldg_stream16(cptr + g * gstride) : make_uint4(0u, 0u, 0u, 0u);
+      if (kSepScales) sb[q] = ok ? ldg_stream8(sptr + g * sgstride) : make_uint2(0u, 0u);
     }
-    return;
-  }
+  };
 
-  // ---------------- consumers
   pdl_wait();  // x, y and the workspace may belong to the previous kernel until here
-  const uint32_t lanereg = tbase | static_cast<uint32_t>(lane * 4);
-  // per-lane address steps: moving row (g ^ lane) by bit b changes the address by +-pitch*2^b
-  constexpr int kSPitch = T::kScaleBox ? 2 * T::kScaleBox : T::kPitch;
-  const Steps dw(lane, T::kPitch), ds(lane, kSPitch);
-  const uint32_t w_off = static_cast<uint32_t>(T::kPitch * lane + 4 * lane);
-  const uint32_t s_off =
-      // (ternary lanes 28..31 hold no words; they read block 3's scale, which is finite
-      // or zero-filled, so that 0 * scale stays 0)
-      FMT == LBQ_TERN5 ? static_cast<uint32_t>(T::kPitch * lane + 28 * (lane / 7 < 3 ? lane / 7 : 3) + 26)
-                       : static_cast<uint32_t>(kStageCodes + kSPitch * lane +
-                                               2 * (lane / (FMT == LBQ_SIGN1 ? 4 : 2)));
+#pragma unroll
+  for (int i = 0; i < kAhead; ++i) load(buf[i], sbuf[i], u_lo + warp + kWarps * i);
   build_slice<FMT>(a, j, tbase, xs, tid);
 
-  bool ok = true;
-  // this warp's units: k = warp, warp + kConsumers, ... (stage k % kStages)
-  for (int32_t k = warp; k < n_units; k += kConsumers) {
-    const int s = k % kStages;
-    const uint32_t use = static_cast<uint32_t>(k / kStages);
-    const uint32_t stage = stage_addr(s);
-    float acc[kRows];
-    if (ok) ok = mbar_wait(full0 + 8 * s, use & 1, a.fault, kFaultConsumer);
-    if (ok) {
-      uint32_t wa = stage + w_off, sa = stage + s_off;
-      // Gray-code walk over g; row (g ^ lane); two rows per step pair
+  const uint32_t lanereg = tbase | static_cast<uint32_t>(lane * 4);
+  const int src6 = (lane & ~7) | 6;  // ternary: the lane holding this block's scale word
+  for (int32_t k = warp; k < n_units; k += kWarps * kAhead) {
 #pragma unroll
-      for (int t = 0; t < kRows; t += 2) {
-        const int g0 = t ^ (t >> 1), g1 = (t + 1) ^ ((t + 1) >> 1);
-        const uint32_t wd0 = lds_u32(wa), sc0 = lds_u16(sa);
-        // step t -> t+1 flips bit 0 of g
-        const int sg0 = (g0 & 1) ? -1 : 1;
-        const uint32_t wa1 = wa + sg0 * dw.at(0), sa1 = sa + sg0 * ds.at(0);
-        const uint32_t wd1 = lds_u32(wa1), sc1 = lds_u16(sa1);
-        const float2 p = lookup4x2(wd0, wd1, lanereg);
-        const float2 sc = make_float2(f16_bits_to_f32(sc0), f16_bits_to_f32(sc1));
-        const float2 r = __fmul2_rn(p, sc);
-        acc[g0] = r.x;
-        acc[g1] = r.y;
-        if (t + 2 < kRows) {  // step t+1 -> t+2 flips bit ctz(t+2) of g
-          const int b = __ffs(t + 2) - 1;
-          const int sg = ((g1 >> b) & 1) ? -1 : 1;
-          wa = wa1 + sg * dw.at(b);
-          sa = sa1 + sg * ds.at(b);
+    for (int i = 0; i < kAhead; ++i) {
+      const int32_t kk = k + kWarps * i;
+      if (kk >= n_units) break;
+      float acc[kRows];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 v = buf[i][q];
+        float2 p01 = lookup_pair(v.x, v.y, lanereg);
+        float2 p23 = lookup_pair(v.z, v.w, lanereg);
+        uint32_t s01, s23;
+        if (kSepScales) {
+          s01 = sbuf[i][q].x;
+          s23 = sbuf[i][q].y;
+        } else {
+          s01 = __shfl_sync(0xffffffffu, __byte_perm(v.x, v.y, 0x7632), src6);
+          s23 = __shfl_sync(0xffffffffu, __byte_perm(v.z, v.w, 0x7632), src6);
+        }
+        p01 = __fmul2_rn(p01, h2_to_f2(s01));
+        p23 = __fmul2_rn(p23, h2_to_f2(s23));
+        acc[4 * q] = p01.x;
+        acc[4 * q + 1] = p01.y;
+        acc[4 * q + 2] = p23.x;
+        acc[4 * q + 3] = p23.y;
+      }
+      load(buf[i], sbuf[i], u_lo + kk + kWarps * kAhead);
+      // transpose-reduce: afterwards acc[0] is row (lane & 15), summed over all lanes
+#pragma unroll
+      for (int d = kRows / 2; d >= 1; d >>= 1) {
+        const bool up = (lane & d) != 0;
+#pragma unroll
+        for (int r = 0; r < d; ++r) {
+          const float send = up ? acc[r] : acc[r + d];
+          const float keep = up ? acc[r + d] : acc[r];
+          acc[r] = keep + __shfl_xor_sync(0xffffffffu, send, d);
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty0 + 8 * s);
-    } else {
-#pragma unroll
-      for (int i = 0; i < kRows; ++i) acc[i] = 0.0f;
-    }
-    // butterfly: acc[i] holds row (i ^ lane); after it, acc[0] is row `lane`
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-#pragma unroll
-      for (int i = 0; i < o; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i + o], o);
-    }
-    if (!ok) continue;
-    const int64_t r = static_cast<int64_t>(c_lo + k) * kRows + lane;
-    if (r < a.N) {
-      if (a.KS == 1)
-        a.y[r] = f32_to_bf16_bits(acc[0]);
-      else
-        a.part[static_cast<int64_t>(j) * a.N + r] = acc[0];
+      acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 16);
+      const int64_t row = static_cast<int64_t>(u_lo + kk) * kRows + lane;
+      if (lane < kRows && row < a.N) {
+        if (a.KS == 1)
+          a.y[row] = f32_to_bf16_bits(acc[0]);
+        else
+          a.part[static_cast<int64_t>(j) * a.N + row] = acc[0];
+      }
     }
   }
 }
@@ -489,48 +432,24 @@ int slices_of(const lbq_weights* w) {
   return static_cast<int>((w->K + per - 1) / per);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// 2D map over [rows][inner] elements with a row pitch in bytes; box = (box_inner, 32).
-bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner,
-              uint64_t rows, uint64_t pitch_bytes, uint32_t box_inner) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {inner, rows};
-  const cuuint64_t strides[1] = {pitch_bytes};
-  const cuuint32_t box[2] = {box_inner, static_cast<cuuint32_t>(kRows)};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int FMT>
 cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uint16_t* y, void* ws,
                    cudaStream_t s) {
-  using T = Traits<FMT>;
   static bool configured[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
     cudaError_t e = cudaFuncSetAttribute(gemv_lut_kernel<FMT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(T::kSmem));
+                                         static_cast<int>(kSmem));
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   Args<FMT> a;
+  a.codes = static_cast<const uint8_t*>(w->codes);
+  a.scales = static_cast<const uint16_t*>(w->scales);
+  a.cstride = w->code_stride;
+  a.sstride = w->scale_stride;
   a.K = w->K;
   a.N = w->N;
   a.x = x;
@@ -542,37 +461,23 @@ cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uin
   if (!a.fault) return cudaErrorInvalidDevicePointer;
   a.part = ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + kWsCounterBytes) : nullptr;
 
-  CUtensorMap tc, ts;
-  const uint64_t row_bytes = FMT == LBQ_TERN5 ? static_cast<uint64_t>(a.nblk) * kTernBlockBytes
-                                              : (FMT == LBQ_SIGN1 ? w->K / 8 : w->K / 4);
-  if (!make_map(&tc, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, row_bytes,
-                static_cast<uint64_t>(w->N), static_cast<uint64_t>(w->code_stride), T::kPitch))
-    return cudaErrorInvalidValue;
-  if (T::kScaleBox) {
-    if (!make_map(&ts, w->scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, static_cast<uint64_t>(a.nblk),
-                  static_cast<uint64_t>(w->N), static_cast<uint64_t>(w->scale_stride) * 2,
-                  T::kScaleBox))
-      return cudaErrorInvalidValue;
-  } else {
-    ts = tc;  // unused
-  }
-  const int64_t NC = (w->N + kRows - 1) / kRows;
+  const int64_t NU = (w->N + kRows - 1) / kRows;
   // Each CTA works on one slice only (one table build): floor(SMs / KS) CTAs per slice.
   const int64_t per = sm_count() / a.KS > 1 ? sm_count() / a.KS : 1;
-  a.G = static_cast<int>(per < NC ? per : NC);
+  a.G = static_cast<int>(per < NU ? per : NU);
   const int64_t grid = static_cast<int64_t>(a.KS) * a.G;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(32 * (T::kConsumers + 1));
-  cfg.dynamicSmemBytes = T::kSmem;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_lut_kernel<FMT>, tc, ts, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_lut_kernel<FMT>, a);
   if (e != cudaSuccess || a.KS == 1) return e;
   cudaLaunchConfig_t cfg2 = cfg;
   cfg2.gridDim = dim3(static_cast<unsigned>((w->N + 255) / 256));

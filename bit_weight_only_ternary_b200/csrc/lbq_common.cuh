@@ -26,6 +26,18 @@ constexpr int64_t kMaxSplitRows = static_cast<int64_t>(kWsCounterBytes / 4) * 32
 // 2^-4.5 = 1/sqrt(512), rounded to fp32.
 constexpr float kRhtNorm = 0.044194173824159216f;
 
+// Storage order shared by every format: rows are interleaved in groups of four. In
+// group g (rows 4g .. 4g+3), 32-bit word w of row 4g+q sits at byte 16 w + 4 q of the
+// group's 4 * code_stride bytes, and scale e of row 4g+q at element 4 e + q of its
+// 4 * scale_stride fp16. One 16-byte load then brings the same word of four rows.
+__host__ __device__ __forceinline__ int64_t g4_rows(int64_t N) { return (N + 3) / 4 * 4; }
+__host__ __device__ __forceinline__ int64_t g4_word_byte(int64_t n, int64_t w, int64_t stride) {
+  return (n >> 2) * 4 * stride + w * 16 + (n & 3) * 4;
+}
+__host__ __device__ __forceinline__ int64_t g4_scale_elem(int64_t n, int64_t e, int64_t sstride) {
+  return (n >> 2) * 4 * sstride + e * 4 + (n & 3);
+}
+
 struct Layout {
   int64_t code_stride;   // bytes per row of codes
   int64_t scale_stride;  // fp16 scales per row (0: scales in-block)

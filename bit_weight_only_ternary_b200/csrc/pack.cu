@@ -43,41 +43,48 @@ __device__ __forceinline__ int trit_of(float w, float half_s, bool zero_scale) {
   return a > half_s ? (w > 0.0f ? 1 : -1) : 0;
 }
 
+// One thread per (row, block) over the rows padded to a multiple of four; padding
+// rows are written as zeros. Codes and scales go to their group-of-four places.
 __global__ void pack_tern_kernel(const float* __restrict__ W, int64_t K, int64_t N,
                                  uint8_t* __restrict__ codes, int64_t stride) {
   const int64_t nb = K / kTernBlock;
   const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (gid >= N * nb) return;
+  if (gid >= g4_rows(N) * nb) return;
   const int64_t n = gid / nb, b = gid % nb;
-  const float* w = W + n * K + b * kTernBlock;
-  const uint16_t h = scale_to_f16_bits(abs_sum<kTernBlock>(w) / 128.0);
-  const float s = f16_bits_to_f32(h);
-  const float half_s = 0.5f * s;
-  const bool zs = (s == 0.0f);
-  uint8_t* out = codes + n * stride + b * kTernBlockBytes;
-  uint8_t bytes[kTernBlockBytes];
+  uint32_t o32[7] = {0, 0, 0, 0, 0, 0, 0};
+  if (n < N) {
+    const float* w = W + n * K + b * kTernBlock;
+    const uint16_t h = scale_to_f16_bits(abs_sum<kTernBlock>(w) / 128.0);
+    const float s = f16_bits_to_f32(h);
+    const float half_s = 0.5f * s;
+    const bool zs = (s == 0.0f);
+    uint8_t bytes[kTernBlockBytes];
 #pragma unroll
-  for (int j = 0; j < kTernCodeBytes; ++j) {
-    int v = 0, p = 1;
+    for (int j = 0; j < kTernCodeBytes; ++j) {
+      int v = 0, p = 1;
 #pragma unroll
-    for (int i = 0; i < 5; ++i) {
-      const int k = 5 * j + i;
-      const int d = (k < kTernBlock) ? trit_of(w[k], half_s, zs) + 1 : 1;
-      v += d * p;
-      p *= 3;
+      for (int i = 0; i < 5; ++i) {
+        const int k = 5 * j + i;
+        const int d = (k < kTernBlock) ? trit_of(w[k], half_s, zs) + 1 : 1;
+        v += d * p;
+        p *= 3;
+      }
+      bytes[j] = static_cast<uint8_t>(v);
     }
-    bytes[j] = static_cast<uint8_t>(v);
+    bytes[26] = static_cast<uint8_t>(h & 0xff);
+    bytes[27] = static_cast<uint8_t>(h >> 8);
+#pragma unroll
+    for (int q = 0; q < 7; ++q)
+      o32[q] = bytes[4 * q] | (bytes[4 * q + 1] << 8) | (bytes[4 * q + 2] << 16) |
+               (static_cast<uint32_t>(bytes[4 * q + 3]) << 24);
   }
-  bytes[26] = static_cast<uint8_t>(h & 0xff);
-  bytes[27] = static_cast<uint8_t>(h >> 8);
-  // the block starts at a multiple of 28 bytes: 4-byte aligned
-  uint32_t* o32 = reinterpret_cast<uint32_t*>(out);
+  // block b is words 7b .. 7b+6 of the row
 #pragma unroll
   for (int q = 0; q < 7; ++q)
-    o32[q] = bytes[4 * q] | (bytes[4 * q + 1] << 8) | (bytes[4 * q + 2] << 16) |
-             (static_cast<uint32_t>(bytes[4 * q + 3]) << 24);
+    *reinterpret_cast<uint32_t*>(codes + g4_word_byte(n, 7 * b + q, stride)) = o32[q];
   if (b == nb - 1)  // zero the row padding
-    for (int64_t p = nb * kTernBlockBytes; p < stride; ++p) codes[n * stride + p] = 0;
+    for (int64_t q = 7 * nb; q < stride / 4; ++q)
+      *reinterpret_cast<uint32_t*>(codes + g4_word_byte(n, q, stride)) = 0u;
 }
 
 __global__ void pack_sign_kernel(const float* __restrict__ W, int64_t K, int64_t N,
@@ -85,20 +92,25 @@ __global__ void pack_sign_kernel(const float* __restrict__ W, int64_t K, int64_t
                                  uint16_t* __restrict__ scales, int64_t sstride) {
   const int64_t nb = K / kSignBlock;
   const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (gid >= N * nb) return;
+  if (gid >= g4_rows(N) * nb) return;
   const int64_t n = gid / nb, b = gid % nb;
-  const float* w = W + n * K + b * kSignBlock;
-  scales[n * sstride + b] = scale_to_f16_bits(abs_sum<kSignBlock>(w) / 128.0);
+  const bool real = n < N;
+  const float* w = W + (real ? n : 0) * K + b * kSignBlock;
+  scales[g4_scale_elem(n, b, sstride)] = real ? scale_to_f16_bits(abs_sum<kSignBlock>(w) / 128.0) : 0;
   if (b == nb - 1)  // zero the scale-row padding
-    for (int64_t p = nb; p < sstride; ++p) scales[n * sstride + p] = 0;
-  uint32_t* o32 = reinterpret_cast<uint32_t*>(codes + n * cstride + b * 16);
+    for (int64_t p = nb; p < sstride; ++p) scales[g4_scale_elem(n, p, sstride)] = 0;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     uint32_t word = 0;
+    if (real) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) word |= (w[32 * q + i] >= 0.0f ? 1u : 0u) << i;
-    o32[q] = word;
+      for (int i = 0; i < 32; ++i) word |= (w[32 * q + i] >= 0.0f ? 1u : 0u) << i;
+    }
+    *reinterpret_cast<uint32_t*>(codes + g4_word_byte(n, 4 * b + q, cstride)) = word;
   }
+  if (b == nb - 1)
+    for (int64_t q = 4 * nb; q < cstride / 4; ++q)
+      *reinterpret_cast<uint32_t*>(codes + g4_word_byte(n, q, cstride)) = 0u;
 }
 
 __global__ void pack_q2_kernel(const float* __restrict__ W, int64_t K, int64_t N,
@@ -106,28 +118,37 @@ __global__ void pack_q2_kernel(const float* __restrict__ W, int64_t K, int64_t N
                                uint16_t* __restrict__ scales, int64_t sstride) {
   const int64_t nb = K / kQ2Block;
   const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (gid >= N * nb) return;
+  if (gid >= g4_rows(N) * nb) return;
   const int64_t n = gid / nb, b = gid % nb;
-  const float* w = W + n * K + b * kQ2Block;
+  const bool real = n < N;
+  const float* w = W + (real ? n : 0) * K + b * kQ2Block;
   float mx = 0.0f;
+  if (real) {
 #pragma unroll
-  for (int i = 0; i < kQ2Block; ++i) mx = fmaxf(mx, fabsf(w[i]));
-  const uint16_t h = scale_to_f16_bits(static_cast<double>(mx) / 1.5);
-  scales[n * sstride + b] = h;
+    for (int i = 0; i < kQ2Block; ++i) mx = fmaxf(mx, fabsf(w[i]));
+  }
+  const uint16_t h = real ? scale_to_f16_bits(static_cast<double>(mx) / 1.5) : 0;
+  scales[g4_scale_elem(n, b, sstride)] = h;
+  if (b == nb - 1)
+    for (int64_t p = nb; p < sstride; ++p) scales[g4_scale_elem(n, p, sstride)] = 0;
   const float s = f16_bits_to_f32(h);
-  uint32_t* o32 = reinterpret_cast<uint32_t*>(codes + n * cstride + b * 8);
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     uint32_t word = 0;
+    if (real) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float v = w[16 * q + i];
-      // nearest of {-1.5,-0.5,0.5,1.5}*s, ties upward: boundaries at -s, 0, s
-      uint32_t c = (s == 0.0f) ? 2u : (v < -s ? 0u : (v < 0.0f ? 1u : (v < s ? 2u : 3u)));
-      word |= c << (2 * i);
+      for (int i = 0; i < 16; ++i) {
+        const float v = w[16 * q + i];
+        // nearest of {-1.5,-0.5,0.5,1.5}*s, ties upward: boundaries at -s, 0, s
+        uint32_t c = (s == 0.0f) ? 2u : (v < -s ? 0u : (v < 0.0f ? 1u : (v < s ? 2u : 3u)));
+        word |= c << (2 * i);
+      }
     }
-    o32[q] = word;
+    *reinterpret_cast<uint32_t*>(codes + g4_word_byte(n, 2 * b + q, cstride)) = word;
   }
+  if (b == nb - 1)
+    for (int64_t q = 2 * nb; q < cstride / 4; ++q)
+      *reinterpret_cast<uint32_t*>(codes + g4_word_byte(n, q, cstride)) = 0u;
 }
 
 __global__ void unpack_kernel(int32_t fmt, const uint8_t* __restrict__ codes, int64_t cstride,
@@ -139,29 +160,32 @@ __global__ void unpack_kernel(int32_t fmt, const uint8_t* __restrict__ codes, in
   if (gid >= N * nb) return;
   const int64_t n = gid / nb, b = gid % nb;
   int8_t* o = out + n * K + b * blk;
-  const uint8_t* c = codes + n * cstride;
+  // byte j of row n (group-of-four order)
+  auto byte_at = [&](int64_t j) -> unsigned {
+    return codes[g4_word_byte(n, j >> 2, cstride) + (j & 3)];
+  };
   float s;
   if (fmt == LBQ_TERN5) {
-    const uint8_t* p = c + b * kTernBlockBytes;
-    s = f16_bits_to_f32(static_cast<uint16_t>(p[26] | (p[27] << 8)));
+    const int64_t p = b * kTernBlockBytes;
+    s = f16_bits_to_f32(static_cast<uint16_t>(byte_at(p + 26) | (byte_at(p + 27) << 8)));
     for (int j = 0; j < kTernCodeBytes; ++j) {
-      unsigned v = p[j];
+      unsigned v = byte_at(p + j);
       for (int i = 0; i < 5 && 5 * j + i < kTernBlock; ++i) {
         o[5 * j + i] = static_cast<int8_t>(static_cast<int>(v % 3u) - 1);
         v /= 3u;
       }
     }
   } else if (fmt == LBQ_SIGN1) {
-    s = f16_bits_to_f32(scales[n * sstride + b]);
+    s = f16_bits_to_f32(scales[g4_scale_elem(n, b, sstride)]);
     for (int i = 0; i < kSignBlock; ++i) {
       const int64_t k = b * kSignBlock + i;
-      o[i] = ((c[k >> 3] >> (k & 7)) & 1) ? 1 : -1;
+      o[i] = ((byte_at(k >> 3) >> (k & 7)) & 1) ? 1 : -1;
     }
   } else {
-    s = f16_bits_to_f32(scales[n * sstride + b]);
+    s = f16_bits_to_f32(scales[g4_scale_elem(n, b, sstride)]);
     for (int i = 0; i < kQ2Block; ++i) {
       const int64_t k = b * kQ2Block + i;
-      o[i] = static_cast<int8_t>((c[k >> 2] >> (2 * (k & 3))) & 3);
+      o[i] = static_cast<int8_t>((byte_at(k >> 2) >> (2 * (k & 3))) & 3);
     }
   }
   if (sout) sout[n * nb + b] = s;
@@ -188,7 +212,7 @@ inline unsigned grid_for(int64_t n, int threads) {
 cudaError_t lbq_launch_pack(int32_t fmt, const float* W, int64_t K, int64_t N, uint8_t* codes,
                             uint16_t* scales, const lbq::Layout& L, cudaStream_t s) {
   const int T = 128;
-  const int64_t units = N * (K / L.block);
+  const int64_t units = g4_rows(N) * (K / L.block);
   switch (fmt) {
     case LBQ_TERN5:
       pack_tern_kernel<<<grid_for(units, T), T, 0, s>>>(W, K, N, codes, L.code_stride);

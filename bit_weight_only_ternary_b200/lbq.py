@@ -100,7 +100,8 @@ def lbq_packed_layout(fmt: int, K: int, N: int):
 
 @dataclass
 class PackedWeights:
-    """A packed matrix: codes uint8 [N][code_stride] and (sign, 2-bit) fp16 scales."""
+    """A packed matrix in the library's group-of-four row order: codes uint8
+    [ceil(N/4)][4 * code_stride] and (sign, 2-bit) fp16 scales [ceil(N/4)][4 * scale_stride]."""
     fmt: int
     K: int
     N: int
@@ -110,7 +111,8 @@ class PackedWeights:
     def desc(self) -> lbq_weights:
         return lbq_weights(self.fmt, 0, self.K, self.N, self.codes.data_ptr(),
                            None if self.scales is None else self.scales.data_ptr(),
-                           self.codes.stride(0), 0 if self.scales is None else self.scales.stride(0))
+                           self.codes.stride(0) // 4,
+                           0 if self.scales is None else self.scales.stride(0) // 4)
 
     @property
     def nbytes(self) -> int:
@@ -122,8 +124,9 @@ def lbq_pack(fmt: int, W: torch.Tensor, stream=None) -> PackedWeights:
     assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous() and W.dim() == 2
     N, K = W.shape
     cs, ss, cb, sb = lbq_packed_layout(fmt, K, N)
-    codes = torch.empty((N, cs), dtype=torch.uint8, device=W.device)
-    scales = torch.empty((N, ss), dtype=torch.int16, device=W.device) if ss else None
+    G = (N + 3) // 4  # rows are stored in groups of four
+    codes = torch.empty((G, 4 * cs), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((G, 4 * ss), dtype=torch.int16, device=W.device) if ss else None
     # (torch's allocations are 256-byte aligned, as the scales' TMA rows require)
     _check(_lib.lbq_pack(fmt, _ptr(W), K, N, _ptr(codes), _ptr(scales), _stream(stream)),
            "lbq_pack")

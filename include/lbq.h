@@ -65,6 +65,15 @@
  *     The weights are expressed in the rotated basis, so the product uses
  *     x' = H_512 D x / sqrt(512) (see lbq_hadamard) in place of x. K % 512 == 0.
  *
+ * Storage order (all formats). The per-row byte strings above are stored with rows
+ *   interleaved in groups of four, so that one 16-byte load brings the same 32-bit
+ *   word of four rows. N is padded to a multiple of four with zero rows. In group g
+ *   (rows 4g .. 4g+3) the group's codes take 4 * code_stride bytes starting at byte
+ *   g * 4 * code_stride, and 32-bit word w of row 4g+q (its bytes 4w .. 4w+3) sits at
+ *   bytes 16 w + 4 q of the group. Scales likewise: the group's 4 * scale_stride fp16
+ *   start at element g * 4 * scale_stride, and scale e of row 4g+q is element 4 e + q
+ *   of the group. Padding rows and padding words are zero bytes.
+ *
  * Shape rules: K % 128 == 0 (LBQ_Q2RHT: K % 512 == 0), K >= 128, N >= 1, M >= 1;
  * a batch-1 product split over K (K > 512, or > 1024 for LBQ_SIGN1) has N <= 524288.
  * Alignment rules: codes, scales, x/X, W, D, out and workspace 16-byte aligned;
@@ -105,10 +114,11 @@ typedef struct lbq_weights {
   int32_t reserved;      /* must be 0                                             */
   int64_t K;             /* input features (packed along a row)                   */
   int64_t N;             /* output features (rows)                                */
-  const void* codes;     /* device, [N][code_stride] bytes                        */
-  const void* scales;    /* device, [N][scale_stride] fp16; NULL for LBQ_TERN5    */
-  int64_t code_stride;   /* bytes between rows of codes                           */
-  int64_t scale_stride;  /* fp16 elements between rows of scales (0 for TERN5)    */
+  const void* codes;     /* device, ceil(N/4) groups of 4*code_stride bytes        */
+  const void* scales;    /* device, ceil(N/4) groups of 4*scale_stride fp16;       *
+                          * NULL for LBQ_TERN5                                     */
+  int64_t code_stride;   /* code bytes per row (a group holds four rows)           */
+  int64_t scale_stride;  /* fp16 scales per row (0 for TERN5)                      */
 } lbq_weights;
 
 /* Human-readable name of a status. Never NULL. Host only. */
@@ -116,14 +126,16 @@ const char* lbq_status_string(lbq_status st);
 
 /* Packed sizes for a K x N matrix in format `fmt` (host only, no CUDA call).
  * Any output pointer may be NULL. code_stride/scale_stride are the minimal
- * strides; code_bytes = N * code_stride, scale_bytes = N * scale_stride * 2.
+ * strides; with N4 = N rounded up to a multiple of four (the storage order groups
+ * rows in fours), code_bytes = N4 * code_stride, scale_bytes = N4 * scale_stride * 2.
  * Errors: LBQ_ERR_FORMAT, LBQ_ERR_SHAPE. */
 lbq_status lbq_packed_layout(int32_t fmt, int64_t K, int64_t N, int64_t* code_stride,
                              int64_t* scale_stride, size_t* code_bytes, size_t* scale_bytes);
 
 /* Quantise and pack W (device fp32 [N][K], row-major, 16-byte aligned) into
- * `codes` ([N][code_stride] bytes) and `scales` ([N][scale_stride] fp16; NULL for
- * TERN5), using the minimal strides of lbq_packed_layout. Rule per format: see the
+ * `codes` (code_bytes) and `scales` (scale_bytes; NULL for TERN5) in the
+ * group-of-four storage order, using the minimal strides of lbq_packed_layout;
+ * padding rows and words are written as zeros. Rule per format: see the
  * header comment ([tern] §5.1 applied per block as in [block] §2.1; [sign]; [rht]).
  * Deterministic and bit-exact: the same W always gives the same bytes. Offline
  * step, not tuned for speed. */

@@ -46,9 +46,10 @@ def test_status_strings(L):
 def test_layout_matches_oracle_layout(L, orc):
     for fmt in (1, 2, 3):
         for K in (512, 1024, 5120, 17408):
-            cs, ss, cb, sb = L.lbq_packed_layout(fmt, K, 3)
-            ocs, oss, _ = orc.layout(fmt, K)
-            assert (cs, ss, cb, sb) == (ocs, oss, 3 * ocs, 3 * oss * 2)
+            for N, N4 in ((3, 4), (4, 4), (9, 12)):  # rows are stored in groups of four
+                cs, ss, cb, sb = L.lbq_packed_layout(fmt, K, N)
+                ocs, oss, _ = orc.layout(fmt, K)
+                assert (cs, ss, cb, sb) == (ocs, oss, N4 * ocs, N4 * oss * 2)
     assert L.lbq_packed_layout(1, 128, 1)[0] == 32
     assert L.lbq_packed_layout(1, 384, 1)[0] == 96  # 3 x 28 = 84 -> 96
 

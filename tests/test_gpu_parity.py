@@ -34,14 +34,16 @@ def _pack_both(L, orc, fmt, W_cpu):
     return pw, codes, scales
 
 
-def _assert_codes_equal(pw, codes, scales):
+def _assert_codes_equal(orc, pw, codes, scales):
+    """The library's buffers against the oracle's rows put in group-of-four order."""
     got = pw.codes.cpu().numpy()
-    assert got.shape == codes.shape
-    bad = np.argwhere(got != codes)
+    want = orc.group4(codes)
+    assert got.shape == want.shape
+    bad = np.argwhere(got != want)
     assert bad.size == 0, f"{len(bad)} code bytes differ, first at {bad[:4].tolist()}"
     if scales is not None:
         gs = pw.scales.cpu().numpy().view(np.uint16)
-        assert np.array_equal(gs, scales), "scales differ"
+        assert np.array_equal(gs, orc.group4(scales)), "scales differ"
 
 
 def _check_products(y, Y, B, what=""):
@@ -74,7 +76,7 @@ SHAPES = [(256, 512), (37, 1536), (1, 512), (5, 1024)]
 def test_pack_bit_exact(L, orc, fmt, N, K):
     W = synth.weights(N, K, 1000 + N + K)
     pw, codes, scales = _pack_both(L, orc, fmt, W)
-    _assert_codes_equal(pw, codes, scales)
+    _assert_codes_equal(orc, pw, codes, scales)
 
 
 @pytest.mark.parametrize("fmt", (TERN5, SIGN1))
@@ -82,7 +84,7 @@ def test_pack_bit_exact(L, orc, fmt, N, K):
 def test_pack_ragged_k_and_row_padding(L, orc, fmt, K):
     W = synth.weights(9, K, 5 + K)
     pw, codes, scales = _pack_both(L, orc, fmt, W)
-    _assert_codes_equal(pw, codes, scales)
+    _assert_codes_equal(orc, pw, codes, scales)
 
 
 @pytest.mark.parametrize("fmt", FMTS)
@@ -98,7 +100,7 @@ def test_pack_adversarial_values(L, orc, fmt):
     W[4, ::2] = -W[4, 1::2]                      # exact +- pairs
     W[5, 32:64] = torch.tensor([-1.5, -1.0, -0.5, 0.0, 0.5, 1.0, 1.5, -1.0] * 4)  # 2-bit ties
     pw, codes, scales = _pack_both(L, orc, fmt, W)
-    _assert_codes_equal(pw, codes, scales)
+    _assert_codes_equal(orc, pw, codes, scales)
 
 
 @pytest.mark.parametrize("fmt", FMTS)
@@ -117,11 +119,13 @@ def test_pack_sampled_rows_of_27b_gate_up(L, orc, fmt):
     N, K = 2 * synth.FFN, synth.HIDDEN
     Wd = synth.weights(N, K, 31337, device="cuda")
     pw = L.lbq_pack(fmt, Wd)
-    rows = torch.tensor([0, 1, 777, 12345, N // 2, N - 2, N - 1])
+    groups = torch.tensor([0, 1, 777, 3000, N // 8, N // 4 - 2, N // 4 - 1])  # groups of 4 rows
+    rows = (4 * groups[:, None] + torch.arange(4)[None, :]).reshape(-1)
     codes, scales = orc.pack(fmt, Wd[rows.cuda()].cpu().numpy())
-    assert np.array_equal(pw.codes[rows.cuda()].cpu().numpy(), codes)
+    assert np.array_equal(pw.codes[groups.cuda()].cpu().numpy(), orc.group4(codes))
     if scales is not None:
-        assert np.array_equal(pw.scales[rows.cuda()].cpu().numpy().view(np.uint16), scales)
+        assert np.array_equal(pw.scales[groups.cuda()].cpu().numpy().view(np.uint16),
+                              orc.group4(scales))
 
 
 # ----------------------------------------------------------------------------- rotation
@@ -165,7 +169,7 @@ def test_gemv_one_27b_layer(L, orc, fmt):
         pw = L.lbq_pack(fmt, Wd)
         codes, scales = orc.pack(fmt, Wd.cpu().numpy())
         del Wd
-        _assert_codes_equal(pw, codes, scales)
+        _assert_codes_equal(orc, pw, codes, scales)
         x = synth.activations(1, K, synth.seed_of(20, 0, mi), device="cuda")
         y = L.lbq_gemv(pw, x[0], _gpu_D(L, fmt, K))
         Y, B = orc.gemm(fmt, codes, scales, K, synth.bf16_bits(x), _oracle_D(orc, fmt, K),
