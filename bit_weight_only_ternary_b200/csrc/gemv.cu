@@ -23,14 +23,20 @@
 //    shared-memory staging, whose extra write and read would cost shared-memory
 //    bandwidth, the kernel's second bound.
 //  * Reduction. Each lane holds one word's partial sum for each of 16 rows; a
-//    transpose-reduce butterfly (15 shuffles) leaves row l's slice sum in lane l.
+//    transpose-reduce butterfly (16 shuffles) leaves row l's slice sum in lane l.
+//    (Rotating the group order per lane would spare the selects of two stages, but
+//    a warp load then touches four groups instead of one, and the extra sectors
+//    cost more than the selects: measured.)
 //  * Scales. Ternary scales live in word 6 of each 28-byte block: lanes are mapped
 //    so that block b is lanes 8b .. 8b+6, and lane 8b+6 hands each pair of rows'
 //    scales to its block's lanes with one shuffle. 1-bit and 2-bit scales come
 //    with one 8-byte load per lane per four rows (group-of-four scale order).
 //  * Split-K. Slices are spread over CTAs; slice sums go to the workspace and a
-//    small second kernel (programmatic dependent launch) adds each row's slice
-//    sums in slice order and writes bf16 y: results are deterministic.
+//    small second kernel (programmatic dependent launch, resident beside the main
+//    kernel) adds each row's slice sums in slice order and writes bf16 y: results
+//    are deterministic. (Folding that sum into the main kernel, by the last CTA of a
+//    row range or after a meeting of the range's CTAs, measured slower: the tail of
+//    L2 round trips then runs on a handful of SMs.)
 //  * Programmatic dependent launch: before waiting for the previous kernel, each
 //    warp asks L2 to prefetch its first units of weights (a hint only: the loads
 //    that feed the arithmetic are issued after the wait, so weights written by the
@@ -160,51 +166,79 @@ __device__ __forceinline__ float2 lookup_pair(uint32_t w0, uint32_t w1, uint32_t
   return __fadd2_rn(__fadd2_rn(e0, e1), __fadd2_rn(e2, e3));
 }
 
-// Builds the x slice and the lookup table for slice j (all threads).
+// The x slice of slice j, in flight: the loads are issued by x_issue (before the
+// weight loads, so that the table build, which waits for x, is not queued behind
+// them) and stored to shared memory as fp32 by x_store.
+struct XLoad {
+  uint4 v0, v1, d;
+};
+template <int FMT>
+__device__ __forceinline__ XLoad x_issue(const Args<FMT>& a, int32_t j, int tid) {
+  using T = Traits<FMT>;
+  XLoad r{make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+  const int64_t k0 = static_cast<int64_t>(j) * T::kWeights;
+  if (FMT == LBQ_Q2RHT) {
+    if (tid < 32) {  // one warp: 16 activations and 16 signs per lane
+      const uint4* x4 = reinterpret_cast<const uint4*>(a.x + k0 + 16 * tid);
+      r.v0 = x4[0];
+      r.v1 = x4[1];
+      r.d = *reinterpret_cast<const uint4*>(a.D + k0 + 16 * tid);
+    }
+  } else {
+    const int blk0 = j * T::kBlocks;
+    const int nb = a.nblk - blk0 < T::kBlocks ? a.nblk - blk0 : T::kBlocks;
+    // one 16-byte load of 8 activations per thread (x and the slices are 16-byte aligned)
+    if (tid < T::kWeights / 8 && 8 * tid < nb * kTernBlock)
+      r.v0 = __ldg(reinterpret_cast<const uint4*>(a.x + k0) + tid);
+  }
+  return r;
+}
+template <int FMT>
+__device__ __forceinline__ void x_store(const XLoad& r, float* xs, int tid) {
+  using T = Traits<FMT>;
+  if (FMT == LBQ_Q2RHT) {
+    if (tid < 32) {
+      const uint32_t xw[8] = {r.v0.x, r.v0.y, r.v0.z, r.v0.w, r.v1.x, r.v1.y, r.v1.z, r.v1.w};
+      const uint32_t dw[4] = {r.d.x, r.d.y, r.d.z, r.d.w};
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint32_t bits = (i & 1) ? (xw[i >> 1] & 0xffff0000u) : (xw[i >> 1] << 16);
+        const int8_t sgn = static_cast<int8_t>((dw[i >> 2] >> (8 * (i & 3))) & 0xff);
+        const float xv = __uint_as_float(bits);
+        v[i] = sgn < 0 ? -xv : xv;
+      }
+      fwht512_warp(v);
+      float4* d = reinterpret_cast<float4*>(xs + 16 * tid);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        d[q] = make_float4(v[4 * q] * kRhtNorm, v[4 * q + 1] * kRhtNorm, v[4 * q + 2] * kRhtNorm,
+                           v[4 * q + 3] * kRhtNorm);
+    }
+  } else if (tid < T::kWeights / 8) {
+    const uint32_t w[4] = {r.v0.x, r.v0.y, r.v0.z, r.v0.w};
+    float f[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      f[2 * q] = __uint_as_float(w[q] << 16);
+      f[2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
+    }
+    float4* d = reinterpret_cast<float4*>(xs + 8 * tid);
+    d[0] = make_float4(f[0], f[1], f[2], f[3]);
+    d[1] = make_float4(f[4], f[5], f[6], f[7]);
+  }
+}
+
+// Builds the lookup table for slice j from the x slice in shared memory (all threads).
 // Thread t owns table column pair t % 64 (lanes 2c, 2c+1 of one byte slot) and the
 // values v = lo + R * hi for hi = t / 64, t / 64 + 8, ...; everything that does not
 // depend on hi is computed once.
 template <int FMT>
-__device__ __forceinline__ void build_slice(const Args<FMT>& a, int32_t j, uint32_t tbase,
-                                            float* xs, int tid) {
+__device__ __forceinline__ void build_table(const Args<FMT>& a, int32_t j, uint32_t tbase,
+                                            const float* xs, int tid) {
   using T = Traits<FMT>;
   const int blk0 = j * T::kBlocks;
   const int nb = a.nblk - blk0 < T::kBlocks ? a.nblk - blk0 : T::kBlocks;
-  const int nx = FMT == LBQ_Q2RHT ? nb * kQ2Block : nb * kTernBlock;
-  const int64_t k0 = static_cast<int64_t>(j) * T::kWeights;
-  const int lane = tid & 31;
-
-  if (FMT == LBQ_Q2RHT) {
-    if (tid < 32) {
-      float v[16];
-      rht512_warp_load(a.x + k0, a.D + k0, v);
-      float4* d = reinterpret_cast<float4*>(xs + 16 * lane);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-    }
-  } else {
-    // one 16-byte load of 8 activations per thread (x and the slices are 16-byte aligned)
-    for (int i = tid; i < T::kWeights / 8; i += kThreads) {
-      float f[8];
-      if (8 * i < nx) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x + k0) + i);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          f[2 * q] = __uint_as_float(w[q] << 16);
-          f[2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
-        }
-      } else {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) f[q] = 0.0f;
-      }
-      float4* d = reinterpret_cast<float4*>(xs + 8 * i);
-      d[0] = make_float4(f[0], f[1], f[2], f[3]);
-      d[1] = make_float4(f[4], f[5], f[6], f[7]);
-    }
-  }
-  __syncthreads();
-
   const int cp = tid & 63;
   const int slot = cp >> 4, l0 = 2 * (cp & 15);
   float2 xv[T::kDigits];
@@ -282,8 +316,10 @@ __device__ __forceinline__ void build_slice(const Args<FMT>& a, int32_t j, uint3
   __syncthreads();
 }
 
+// At most 120 registers a thread (of the SM's 64 K, 61440 for the 512 threads), so
+// that a CTA of the split-K sum kernel (128 threads x 32) fits beside it.
 template <int FMT>
-__global__ void __launch_bounds__(kThreads, 1) gemv_lut_kernel(const Args<FMT> a) {
+__global__ void __maxnreg__(120) gemv_lut_kernel(const Args<FMT> a) {
   using T = Traits<FMT>;
   constexpr bool kSepScales = FMT != LBQ_TERN5;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -315,9 +351,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_kernel(const Args<FMT> a
   const int wl = lane_word<FMT>(lane, nb);
   const int64_t gstride = 4 * a.cstride;  // bytes per group of four rows
   const uint8_t* slice = a.codes + static_cast<int64_t>(16) * j * T::kWords;
+  // Lanes without a word (their table columns are zero) read word 0 of the slice:
+  // every load is in bounds and none needs a predicate.
   const uint8_t* cptr = slice + 16 * (wl < 0 ? 0 : wl);
   // 1-bit / 2-bit: this lane's block scales of four rows are 8 bytes of the group
-  const int sblk = blk0 + (FMT == LBQ_SIGN1 ? (lane >> 2) : (lane >> 1));
+  // (a lane without a word reads the slice's first block: finite, times zero).
+  const int sblk = wl < 0 ? blk0 : blk0 + (FMT == LBQ_SIGN1 ? (lane >> 2) : (lane >> 1));
   const uint16_t* sptr = kSepScales ? a.scales + 4 * sblk : nullptr;
   const int64_t sgstride = 4 * a.sstride;
 
@@ -332,23 +371,44 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_kernel(const Args<FMT> a
 
   uint4 buf[kAhead][4];
   uint2 sbuf[kAhead][4];
+  // Units past this CTA's range reload its last unit, and groups past the last row
+  // reload the last group: the values are never used.
   auto load = [&](uint4 (&b)[4], uint2 (&sb)[4], int32_t u) {
+    const int32_t uc = u < u_hi ? u : u_hi - 1;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const int32_t g = 4 * u + q;
-      const bool ok = u < u_hi && g < NG && wl >= 0;
-      b[q] = ok ? ldg_stream16(cptr + g * gstride) : make_uint4(0u, 0u, 0u, 0u);
-      if (kSepScales) sb[q] = ok ? ldg_stream8(sptr + g * sgstride) : make_uint2(0u, 0u);
+      int32_t g = 4 * uc + q;
+      g = g < NG ? g : NG - 1;
+      b[q] = ldg_stream16(cptr + static_cast<int64_t>(g) * gstride);
+      if (kSepScales) sb[q] = ldg_stream8(sptr + static_cast<int64_t>(g) * sgstride);
     }
   };
 
+  // ... and for the x slice (written by the previous kernel in a chain of products:
+  // a prefetch into L2 is only a hint and cannot return stale data)
+  if (tid >= 480 && tid - 480 < T::kWeights / 64) {
+    const int64_t k = static_cast<int64_t>(j) * T::kWeights + 64 * (tid - 480);
+    if (k + 64 <= a.K) prefetch_l2_bulk(a.x + k, 128);
+    if (FMT == LBQ_Q2RHT && tid - 480 < T::kWeights / 128)
+      prefetch_l2_bulk(a.D + static_cast<int64_t>(j) * T::kWeights + 128 * (tid - 480), 128);
+  }
+
   pdl_wait();  // x, y and the workspace may belong to the previous kernel until here
+  // x first, alone, then the table: weight loads issued beside them would queue
+  // ahead of them (the first units' weights were prefetched into L2 above)
+  x_store<FMT>(x_issue<FMT>(a, j, tid), xs, tid);
+  __syncthreads();
+  load(buf[0], sbuf[0], u_lo + warp);  // one unit in flight during the build
+  build_table<FMT>(a, j, tbase, xs, tid);
 #pragma unroll
-  for (int i = 0; i < kAhead; ++i) load(buf[i], sbuf[i], u_lo + warp + kWarps * i);
-  build_slice<FMT>(a, j, tbase, xs, tid);
+  for (int i = 1; i < kAhead; ++i) load(buf[i], sbuf[i], u_lo + warp + kWarps * i);
 
   const uint32_t lanereg = tbase | static_cast<uint32_t>(lane * 4);
   const int src6 = (lane & ~7) | 6;  // ternary: the lane holding this block's scale word
+  const int64_t NR = a.N;
+  float* const part_j = a.part + static_cast<int64_t>(j) * NR;
+  uint16_t* const y = a.y;
+  const bool direct = a.KS == 1;
   for (int32_t k = warp; k < n_units; k += kWarps * kAhead) {
 #pragma unroll
     for (int i = 0; i < kAhead; ++i) {
@@ -389,39 +449,41 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_kernel(const Args<FMT> a
       }
       acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 16);
       const int64_t row = static_cast<int64_t>(u_lo + kk) * kRows + lane;
-      if (lane < kRows && row < a.N) {
-        if (a.KS == 1)
-          a.y[row] = f32_to_bf16_bits(acc[0]);
+      if (lane < kRows && row < NR) {
+        if (direct)
+          y[row] = f32_to_bf16_bits(acc[0]);
         else
-          a.part[static_cast<int64_t>(j) * a.N + row] = acc[0];
+          part_j[row] = acc[0];
       }
     }
   }
 }
 
 // Sums the slice sums of every row in slice order and writes bf16 y. Launched right
-// after the main kernel with programmatic dependent launch: it may start while that
-// kernel is finishing and waits for its results before reading them.
-__global__ void __launch_bounds__(256) splitk_sum_kernel(const float* __restrict__ part, int KS,
-                                                         int64_t N, uint16_t* __restrict__ y) {
+// after the main kernel with programmatic dependent launch: its CTAs become resident
+// while that kernel runs (the main kernel leaves room for one per SM) and wait for
+// its results before reading them. Twelve of a row's loads are in flight at once.
+constexpr int kSumThreads = 128;
+__global__ void __maxnreg__(32)
+    splitk_sum_kernel(const float* __restrict__ part,
+                                                                 int KS, int64_t N,
+                                                                 uint16_t* __restrict__ y) {
   pdl_launch_dependents();
   pdl_wait();
-  const int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (r >= N) return;
-  const float* pr = part + r;
-  float sum = 0.0f;
-  // all of a row's loads are issued before the sum (16 slices per round); the
-  // additions then run in slice order
-  for (int j = 0; j < KS; j += 16) {
-    float v[16];
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * kSumThreads + threadIdx.x; r < N;
+       r += static_cast<int64_t>(gridDim.x) * kSumThreads) {
+    float sum = 0.0f;
+    const float* p = part + r;
+    for (int j = 0; j < KS; j += 12) {
+      float v[12];
 #pragma unroll
-    for (int q = 0; q < 16; ++q)
-      v[q] = j + q < KS ? __ldcg(pr + static_cast<int64_t>(j + q) * N) : 0.0f;
+      for (int q = 0; q < 12; ++q) v[q] = j + q < KS ? __ldcg(p + (j + q) * N) : 0.0f;
 #pragma unroll
-    for (int q = 0; q < 16; ++q)
-      if (j + q < KS) sum += v[q];
+      for (int q = 0; q < 12; ++q)
+        if (j + q < KS) sum += v[q];
+    }
+    y[r] = f32_to_bf16_bits(sum);
   }
-  y[r] = f32_to_bf16_bits(sum);
 }
 
 // The device word the kernels' bounded waits report to (one per device).
@@ -480,8 +542,10 @@ cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uin
   cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_lut_kernel<FMT>, a);
   if (e != cudaSuccess || a.KS == 1) return e;
   cudaLaunchConfig_t cfg2 = cfg;
-  cfg2.gridDim = dim3(static_cast<unsigned>((w->N + 255) / 256));
-  cfg2.blockDim = dim3(256);
+  const int64_t rows_per_cta = kSumThreads;
+  const int64_t ctas = (w->N + rows_per_cta - 1) / rows_per_cta;
+  cfg2.gridDim = dim3(static_cast<unsigned>(ctas < sm_count() ? ctas : sm_count()));
+  cfg2.blockDim = dim3(kSumThreads);
   cfg2.dynamicSmemBytes = 0;
   return cudaLaunchKernelEx(&cfg2, splitk_sum_kernel, static_cast<const float*>(a.part), a.KS,
                             static_cast<int64_t>(w->N), y);
