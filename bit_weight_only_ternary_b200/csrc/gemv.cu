@@ -43,6 +43,8 @@
 //    previous kernel are always read correctly).
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include "rht.cuh"
 #include "sm100_async.cuh"
 
@@ -371,16 +373,18 @@ __global__ void __maxnreg__(120) gemv_lut_kernel(const Args<FMT> a) {
 
   uint4 buf[kAhead][4];
   uint2 sbuf[kAhead][4];
-  // Units past this CTA's range reload its last unit, and groups past the last row
-  // reload the last group: the values are never used.
-  auto load = [&](uint4 (&b)[4], uint2 (&sb)[4], int32_t u) {
-    const int32_t uc = u < u_hi ? u : u_hi - 1;
+  // This warp's units: u_lo + warp + kWarps t for t < nt. Groups past the last row
+  // (the matrix's last unit) reload the last group: those rows are never written.
+  const int32_t nt = n_units > warp ? (n_units - warp + kWarps - 1) / kWarps : 0;
+  const uint32_t gstride32 = static_cast<uint32_t>(gstride);
+  const uint32_t sgstride32 = static_cast<uint32_t>(sgstride);
+  auto load = [&](uint4 (&b)[4], uint2 (&sb)[4], int32_t t) {
+    const uint32_t g0 = 4u * static_cast<uint32_t>(u_lo + warp + kWarps * t);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      int32_t g = 4 * uc + q;
-      g = g < NG ? g : NG - 1;
-      b[q] = ldg_stream16(cptr + static_cast<int64_t>(g) * gstride);
-      if (kSepScales) sb[q] = ldg_stream8(sptr + static_cast<int64_t>(g) * sgstride);
+      const uint32_t g = min(g0 + q, static_cast<uint32_t>(NG - 1));
+      b[q] = ldg_stream16(cptr + static_cast<uint64_t>(g) * gstride32);
+      if (kSepScales) sb[q] = ldg_stream8(sptr + static_cast<uint64_t>(g) * sgstride32);
     }
   };
 
@@ -398,10 +402,11 @@ __global__ void __maxnreg__(120) gemv_lut_kernel(const Args<FMT> a) {
   // ahead of them (the first units' weights were prefetched into L2 above)
   x_store<FMT>(x_issue<FMT>(a, j, tid), xs, tid);
   __syncthreads();
-  load(buf[0], sbuf[0], u_lo + warp);  // one unit in flight during the build
+  if (nt > 0) load(buf[0], sbuf[0], 0);  // one unit in flight during the build
   build_table<FMT>(a, j, tbase, xs, tid);
 #pragma unroll
-  for (int i = 1; i < kAhead; ++i) load(buf[i], sbuf[i], u_lo + warp + kWarps * i);
+  for (int i = 1; i < kAhead; ++i)
+    if (i < nt) load(buf[i], sbuf[i], i);
 
   const uint32_t lanereg = tbase | static_cast<uint32_t>(lane * 4);
   const int src6 = (lane & ~7) | 6;  // ternary: the lane holding this block's scale word
@@ -409,80 +414,125 @@ __global__ void __maxnreg__(120) gemv_lut_kernel(const Args<FMT> a) {
   float* const part_j = a.part + static_cast<int64_t>(j) * NR;
   uint16_t* const y = a.y;
   const bool direct = a.KS == 1;
-  for (int32_t k = warp; k < n_units; k += kWarps * kAhead) {
+  // one unit: table lookups, block scales, transpose-reduce, store
+  auto unit = [&](const uint4 (&b)[4], const uint2 (&sb)[4], int32_t t) {
+    float acc[kRows];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 v = b[q];
+      float2 p01 = lookup_pair(v.x, v.y, lanereg);
+      float2 p23 = lookup_pair(v.z, v.w, lanereg);
+      uint32_t s01, s23;
+      if (kSepScales) {
+        s01 = sb[q].x;
+        s23 = sb[q].y;
+      } else {
+        s01 = __shfl_sync(0xffffffffu, __byte_perm(v.x, v.y, 0x7632), src6);
+        s23 = __shfl_sync(0xffffffffu, __byte_perm(v.z, v.w, 0x7632), src6);
+      }
+      p01 = __fmul2_rn(p01, h2_to_f2(s01));
+      p23 = __fmul2_rn(p23, h2_to_f2(s23));
+      acc[4 * q] = p01.x;
+      acc[4 * q + 1] = p01.y;
+      acc[4 * q + 2] = p23.x;
+      acc[4 * q + 3] = p23.y;
+    }
+    // transpose-reduce: afterwards acc[0] is row (lane & 15), summed over all lanes
+#pragma unroll
+    for (int d = kRows / 2; d >= 1; d >>= 1) {
+      const bool up = (lane & d) != 0;
+#pragma unroll
+      for (int r = 0; r < d; ++r) {
+        const float send = up ? acc[r] : acc[r + d];
+        const float keep = up ? acc[r + d] : acc[r];
+        acc[r] = keep + __shfl_xor_sync(0xffffffffu, send, d);
+      }
+    }
+    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 16);
+    const int64_t row = static_cast<int64_t>(u_lo + warp + kWarps * t) * kRows + lane;
+    if (lane < kRows && row < NR) {
+      if (direct)
+        y[row] = f32_to_bf16_bits(acc[0]);
+      else
+        part_j[row] = acc[0];
+    }
+  };
+  int32_t t = 0;
+  for (; t + kAhead <= nt; t += kAhead) {
 #pragma unroll
     for (int i = 0; i < kAhead; ++i) {
-      const int32_t kk = k + kWarps * i;
-      if (kk >= n_units) break;
-      float acc[kRows];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 v = buf[i][q];
-        float2 p01 = lookup_pair(v.x, v.y, lanereg);
-        float2 p23 = lookup_pair(v.z, v.w, lanereg);
-        uint32_t s01, s23;
-        if (kSepScales) {
-          s01 = sbuf[i][q].x;
-          s23 = sbuf[i][q].y;
-        } else {
-          s01 = __shfl_sync(0xffffffffu, __byte_perm(v.x, v.y, 0x7632), src6);
-          s23 = __shfl_sync(0xffffffffu, __byte_perm(v.z, v.w, 0x7632), src6);
-        }
-        p01 = __fmul2_rn(p01, h2_to_f2(s01));
-        p23 = __fmul2_rn(p23, h2_to_f2(s23));
-        acc[4 * q] = p01.x;
-        acc[4 * q + 1] = p01.y;
-        acc[4 * q + 2] = p23.x;
-        acc[4 * q + 3] = p23.y;
-      }
-      load(buf[i], sbuf[i], u_lo + kk + kWarps * kAhead);
-      // transpose-reduce: afterwards acc[0] is row (lane & 15), summed over all lanes
-#pragma unroll
-      for (int d = kRows / 2; d >= 1; d >>= 1) {
-        const bool up = (lane & d) != 0;
-#pragma unroll
-        for (int r = 0; r < d; ++r) {
-          const float send = up ? acc[r] : acc[r + d];
-          const float keep = up ? acc[r + d] : acc[r];
-          acc[r] = keep + __shfl_xor_sync(0xffffffffu, send, d);
-        }
-      }
-      acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 16);
-      const int64_t row = static_cast<int64_t>(u_lo + kk) * kRows + lane;
-      if (lane < kRows && row < NR) {
-        if (direct)
-          y[row] = f32_to_bf16_bits(acc[0]);
-        else
-          part_j[row] = acc[0];
-      }
+      unit(buf[i], sbuf[i], t + i);
+      if (t + i + kAhead < nt) load(buf[i], sbuf[i], t + i + kAhead);
     }
   }
+#pragma unroll
+  for (int i = 0; i < kAhead - 1; ++i)
+    if (t + i < nt) unit(buf[i], sbuf[i], t + i);
 }
 
-// Sums the slice sums of every row in slice order and writes bf16 y. Launched right
-// after the main kernel with programmatic dependent launch: its CTAs become resident
-// while that kernel runs (the main kernel leaves room for one per SM) and wait for
-// its results before reading them. Twelve of a row's loads are in flight at once.
-constexpr int kSumThreads = 128;
+// Sums the slice sums of every row and writes bf16 y. Launched right after the main
+// kernel with programmatic dependent launch: its CTAs become resident while that
+// kernel runs (the main kernel leaves room for one per SM) and wait for its results
+// before reading them. The tail is bound by L2 round trips, so every load of a
+// thread is issued before its adds: a thread takes a pair of rows (one row when N
+// is odd, where pairs would be misaligned) and a run of at most kSumRun slices; the
+// P threads of a row (consecutive lanes) then combine their runs in a fixed tree
+// order, so results are deterministic.
+constexpr int kSumThreads = 128, kSumRun = 8;
+template <bool kPairs>
 __global__ void __maxnreg__(32)
-    splitk_sum_kernel(const float* __restrict__ part,
-                                                                 int KS, int64_t N,
-                                                                 uint16_t* __restrict__ y) {
+    splitk_sum_kernel(const float* __restrict__ part, int KS, int64_t N, int logP,
+                      uint16_t* __restrict__ y) {
   pdl_launch_dependents();
   pdl_wait();
-  for (int64_t r = static_cast<int64_t>(blockIdx.x) * kSumThreads + threadIdx.x; r < N;
-       r += static_cast<int64_t>(gridDim.x) * kSumThreads) {
-    float sum = 0.0f;
-    const float* p = part + r;
-    for (int j = 0; j < KS; j += 12) {
-      float v[12];
+  using V = typename std::conditional<kPairs, float2, float>::type;
+  const int P = 1 << logP;
+  const int run = (KS + P - 1) >> logP;
+  const int64_t nv = kPairs ? N / 2 : N;  // pairs (or rows) per slice
+  const int64_t total = nv << logP;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kSumThreads;
+  // warp-uniform trip count: every lane of a CTA runs the same iterations
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kSumThreads; base < total; base += stride) {
+    const int64_t idx = base + threadIdx.x;
+    const int64_t e = idx >> logP;
+    const int sg = static_cast<int>(idx & (P - 1));
+    const int j0 = sg * run;
+    const int j1 = min(j0 + run, KS);
+    float ax = 0.0f, ay = 0.0f;
+    if (idx < total) {
+      const V* p = reinterpret_cast<const V*>(part) + e;
+      V v[kSumRun];
 #pragma unroll
-      for (int q = 0; q < 12; ++q) v[q] = j + q < KS ? __ldcg(p + (j + q) * N) : 0.0f;
+      for (int q = 0; q < kSumRun; ++q) {
+        if (j0 + q < j1) {
+          v[q] = __ldcg(p + (j0 + q) * nv);
+        } else {
+          v[q] = V{};
+        }
+      }
 #pragma unroll
-      for (int q = 0; q < 12; ++q)
-        if (j + q < KS) sum += v[q];
+      for (int q = 0; q < kSumRun; ++q)
+        if (j0 + q < j1) {
+          if constexpr (kPairs) {
+            ax += v[q].x;
+            ay += v[q].y;
+          } else {
+            ax += v[q];
+          }
+        }
     }
-    y[r] = f32_to_bf16_bits(sum);
+    for (int o = P >> 1; o >= 1; o >>= 1) {
+      ax += __shfl_down_sync(0xffffffffu, ax, o, P);
+      if (kPairs) ay += __shfl_down_sync(0xffffffffu, ay, o, P);
+    }
+    if (idx < total && sg == 0) {
+      if (kPairs) {
+        y[2 * e] = f32_to_bf16_bits(ax);
+        y[2 * e + 1] = f32_to_bf16_bits(ay);
+      } else {
+        y[e] = f32_to_bf16_bits(ax);
+      }
+    }
   }
 }
 
@@ -542,13 +592,18 @@ cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uin
   cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_lut_kernel<FMT>, a);
   if (e != cudaSuccess || a.KS == 1) return e;
   cudaLaunchConfig_t cfg2 = cfg;
-  const int64_t rows_per_cta = kSumThreads;
-  const int64_t ctas = (w->N + rows_per_cta - 1) / rows_per_cta;
+  int logP = 0;
+  while ((a.KS + (1 << logP) - 1) >> logP > kSumRun) ++logP;
+  const bool pairs = (w->N % 2) == 0;
+  const int64_t threads = (pairs ? w->N / 2 : w->N) << logP;
+  const int64_t ctas = (threads + kSumThreads - 1) / kSumThreads;
   cfg2.gridDim = dim3(static_cast<unsigned>(ctas < sm_count() ? ctas : sm_count()));
   cfg2.blockDim = dim3(kSumThreads);
   cfg2.dynamicSmemBytes = 0;
-  return cudaLaunchKernelEx(&cfg2, splitk_sum_kernel, static_cast<const float*>(a.part), a.KS,
-                            static_cast<int64_t>(w->N), y);
+  const float* part = a.part;
+  const int64_t N = w->N;
+  return pairs ? cudaLaunchKernelEx(&cfg2, splitk_sum_kernel<true>, part, a.KS, N, logP, y)
+               : cudaLaunchKernelEx(&cfg2, splitk_sum_kernel<false>, part, a.KS, N, logP, y);
 }
 
 }  // namespace
