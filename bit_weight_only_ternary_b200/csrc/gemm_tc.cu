@@ -43,7 +43,7 @@ using namespace lbq;
 
 constexpr int kTileN = 128;     // weight rows per tile (MMA M)
 constexpr int kTileK = 128;     // K per stage (one ternary block)
-constexpr int kMaxTileM = 128;  // tokens per tile (MMA N)
+constexpr int kMaxTileM = 256;  // tokens per tile (MMA N)
 constexpr int kStagesTC = 4;
 constexpr int kDecoders = 4 * kTileN;  // four threads per weight row, a quarter block each
 constexpr int kThreadsTC = 128 + kDecoders;
@@ -57,7 +57,10 @@ constexpr uint32_t kChunkWords = kChunkBlocks * kTernBlockBytes / 4;
 constexpr uint32_t kGroupWords = 4 * kChunkWords + 4;
 constexpr uint32_t kRawStageBytes = kGroupWords * 4 * (kTileN / 4);
 constexpr int kRawStages = 2;
-constexpr uint32_t kStageB = 2 * kMaxTileM * 128;  // two 64-k slabs of activations
+// Activations arrive in slabs of K = 64 (one 128-byte swizzle row per token), a ring
+// of kSlabs; an A stage (K = 128, one ternary block) consumes two of them.
+constexpr int kSlabs = 4;
+constexpr uint32_t kStageB = kMaxTileM * 128;  // one slab
 // Tensor memory (512 columns): nacc fp32 accumulators of tile_m columns each in
 // [0, 256), the fp16 weight stages at kTmemA + 64 s (128 rows x 128 K = 64 columns
 // each). Successive MMAs go to different accumulators: an MMA that depends on the
@@ -74,7 +77,7 @@ constexpr uint32_t kTmemCols = 512, kTmemA = 256, kAccCols = 256;
 constexpr uint32_t kTabBytes = 243 * 256;
 constexpr uint32_t kLowBytes = 256 + kRawStages * kRawStageBytes + kStageB;
 constexpr uint32_t kHighB = 0xF400;  // first activation stage above the table (1 KB aligned)
-constexpr uint32_t kHighBytes = kHighB + (kStagesTC - 1) * kStageB;
+constexpr uint32_t kHighBytes = kHighB + (kSlabs - 1) * kStageB;
 constexpr size_t kSmemTC = 0x10000 - 0x400 + kHighBytes;
 static_assert(kTabBytes <= kHighB, "table overlaps stage 1");
 static_assert(0x400 + kLowBytes <= 0x10000, "low region does not fit below 64 KB");
@@ -247,8 +250,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const int nkb_all = static_cast<int>(a.K / kTileK);
   const int nkb = (nkb_all - kb0 < a.kb_per_split) ? nkb_all - kb0 : a.kb_per_split;
   const int nchunks = (nkb + kChunkBlocks - 1) / kChunkBlocks;
-  const uint32_t fullA = bars, fullB = fullA + 8 * kStagesTC;
-  const uint32_t empty = fullB + 8 * kStagesTC, accum = empty + 8 * kStagesTC;
+  // fullA / emptyA: tensor-memory weight stages; fullB / emptyB: activation slabs
+  const uint32_t fullA = bars, emptyA = fullA + 8 * kStagesTC;
+  const uint32_t fullB = emptyA + 8 * kStagesTC, emptyB = fullB + 8 * kSlabs;
+  const uint32_t accum = emptyB + 8 * kSlabs;
   const uint32_t fullR = accum + 8, emptyR = fullR + 8 * kRawStages;
   const uint32_t tslot = emptyR + 8 * kRawStages;
   auto bstage = [&](int s) { return s == 0 ? bstage0 : tab + kHighB + (s - 1) * kStageB; };
@@ -257,8 +262,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   if (tid == 0) {
     for (int s = 0; s < kStagesTC; ++s) {
       mbar_init(fullA + 8 * s, kDecoders);  // every decoder thread arrives
+      mbar_init(emptyA + 8 * s, 1);         // the MMA commit arrives
+    }
+    for (int s = 0; s < kSlabs; ++s) {
       mbar_init(fullB + 8 * s, 1);          // the activation TMA lane arrives (+ bytes)
-      mbar_init(empty + 8 * s, 1);          // the MMA commit arrives
+      mbar_init(emptyB + 8 * s, 1);         // the MMA commit arrives
     }
     for (int r = 0; r < kRawStages; ++r) {
       mbar_init(fullR + 8 * r, 1);          // the weight TMA lane arrives (+ bytes)
@@ -278,50 +286,54 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   asm volatile("ld.shared.b32 %0, [%1];" : "=r"(tmem) : "r"(tslot));
 
   if (warp == 0) {
-    // ---------------- activations: two 64-k boxes per stage, 128-byte swizzled
+    // ---------------- activations: one 64-k box per slab, 128-byte swizzled
     if (lane == 0) {
       prefetch_tmap(&tm_x);
-      const uint32_t bytes = 2u * static_cast<uint32_t>(a.tile_m) * 128u;
+      const uint32_t bytes = static_cast<uint32_t>(a.tile_m) * 128u;
+      const int nsl = 2 * nkb;
       int issued = 0;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % kStagesTC;
-        const uint32_t use = static_cast<uint32_t>(kb / kStagesTC);
-        if (!mbar_wait(empty + 8 * s, (use & 1) ^ 1, a.fault, kFaultX)) break;
+      for (int sl = 0; sl < nsl; ++sl) {
+        const int s = sl % kSlabs;
+        const uint32_t use = static_cast<uint32_t>(sl / kSlabs);
+        if (!mbar_wait(emptyB + 8 * s, (use & 1) ^ 1, a.fault, kFaultX)) break;
         ++issued;
         mbar_arrive_expect_tx(fullB + 8 * s, bytes);
-        const uint32_t dst = bstage(s);
-        tma_load_2d(dst, &tm_x, (kb0 + kb) * kTileK, static_cast<int32_t>(m0), fullB + 8 * s);
-        tma_load_2d(dst + static_cast<uint32_t>(a.tile_m) * 128u, &tm_x, (kb0 + kb) * kTileK + 64,
-                    static_cast<int32_t>(m0), fullB + 8 * s);
+        tma_load_2d(bstage(s), &tm_x, kb0 * kTileK + 64 * sl, static_cast<int32_t>(m0), fullB + 8 * s);
       }
       // every issued copy must land before this CTA can exit (matters after a fault)
-      for (int kb = issued - kStagesTC > 0 ? issued - kStagesTC : 0; kb < issued; ++kb)
-        mbar_wait(fullB + 8 * (kb % kStagesTC), static_cast<uint32_t>(kb / kStagesTC) & 1,
+      for (int sl = issued - kSlabs > 0 ? issued - kSlabs : 0; sl < issued; ++sl)
+        mbar_wait(fullB + 8 * (sl % kSlabs), static_cast<uint32_t>(sl / kSlabs) & 1,
                   a.fault, kFaultX, /*give_up_after_fault=*/false);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issue: 8 instructions of K = 16 per stage. The whole warp
-    // runs the loop (so descriptors stay warp-uniform); one elected lane issues.
+    // ---------------- MMA issue: 8 instructions of K = 16 per weight stage, four per
+    // activation slab. The whole warp runs the loop (so descriptors stay
+    // warp-uniform); one elected lane issues.
     const uint32_t idesc = idesc_f16_m128(a.tile_m);
-    const uint32_t slab_b = static_cast<uint32_t>(a.tile_m) * 128u;
     for (int kb = 0; kb < nkb; ++kb) {
       const int s = kb % kStagesTC;
-      const uint32_t par = static_cast<uint32_t>(kb / kStagesTC) & 1;
       bool ok = true;
-      if (lane == 0)
-        ok = mbar_wait(fullA + 8 * s, par, a.fault, kFaultMma) &&
-             mbar_wait(fullB + 8 * s, par, a.fault, kFaultMma);
+      if (lane == 0) ok = mbar_wait(fullA + 8 * s, static_cast<uint32_t>(kb / kStagesTC) & 1, a.fault, kFaultMma);
       if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
-      tc_fence_after_sync();
-      const uint32_t ta = tmem + kTmemA + 64u * s, sb = bstage(s);
+      const uint32_t ta = tmem + kTmemA + 64u * s;
 #pragma unroll
-      for (int ks = 0; ks < kTileK / 16; ++ks) {  // K = 16: 8 tensor-memory columns of A
-        const uint32_t slab = ks >> 2, koff = (ks & 3) * 32;
-        const int i = kb * (kTileK / 16) + ks;    // MMA number; accumulator i % nacc
-        mma_f16_ts_warp(tmem + static_cast<uint32_t>((i & (a.nacc - 1)) * a.tile_m), ta + 8u * ks,
-                        sw128_desc(sb + slab * slab_b + koff), idesc, i >= a.nacc ? 1u : 0u);
+      for (int h = 0; h < 2; ++h) {
+        const int sl = 2 * kb + h, sb_i = sl % kSlabs;
+        if (lane == 0) ok = mbar_wait(fullB + 8 * sb_i, static_cast<uint32_t>(sl / kSlabs) & 1, a.fault, kFaultMma);
+        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+        tc_fence_after_sync();
+        const uint32_t sb = bstage(sb_i);
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {  // K = 16: 8 tensor-memory columns of A, 32 bytes of B
+          const int ks = 4 * h + k4;
+          const int i = kb * (kTileK / 16) + ks;  // MMA number; accumulator i % nacc
+          mma_f16_ts_warp(tmem + static_cast<uint32_t>((i & (a.nacc - 1)) * a.tile_m), ta + 8u * ks,
+                          sw128_desc(sb + 32u * k4), idesc, i >= a.nacc ? 1u : 0u);
+        }
+        mma_commit_warp(emptyB + 8 * sb_i);  // the slab is free once these MMAs are done
       }
-      mma_commit_warp(empty + 8 * s);  // the stage is free once these MMAs are done
+      if (!ok) break;
+      mma_commit_warp(emptyA + 8 * s);  // and the weight stage once all eight are
     }
     mma_commit_warp(accum);  // the accumulator is complete once every MMA is done
   } else if (warp == 2) {
@@ -361,7 +373,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     // store block kb once the MMA has released its stage; completes during the next decode
     auto store = [&]() {
       const int s = kb % kStagesTC;
-      if (ok) ok = mbar_wait(empty + 8 * s, (static_cast<uint32_t>(kb / kStagesTC) & 1) ^ 1, a.fault,
+      if (ok) ok = mbar_wait(emptyA + 8 * s, (static_cast<uint32_t>(kb / kStagesTC) & 1) ^ 1, a.fault,
                              kFaultDecode);
       __syncwarp();  // tcgen05.st is warp-collective
       tc_fence_after_sync();
@@ -495,8 +507,14 @@ struct TcPlan {
 // cannot fill the SMs (small batches).
 TcPlan plan_for(const lbq_weights* w, int64_t M) {
   TcPlan p;
-  p.tile_m = M >= kMaxTileM ? kMaxTileM : static_cast<int>((M + 15) / 16 * 16);
-  const int64_t tiles = ((w->N + kTileN - 1) / kTileN) * ((M + p.tile_m - 1) / p.tile_m);
+  // 256 tokens per tile (the widest MMA, which also hides an MMA's latency behind the
+  // next) unless that leaves SMs idle, then 128; small batches round up to 16.
+  const int64_t ntiles = (w->N + kTileN - 1) / kTileN;
+  if (M >= 256 && ntiles * ((M + 255) / 256) >= sm_count())
+    p.tile_m = 256;
+  else
+    p.tile_m = M >= 128 ? 128 : static_cast<int>((M + 15) / 16 * 16);
+  const int64_t tiles = ntiles * ((M + p.tile_m - 1) / p.tile_m);
   const int nkb = static_cast<int>(w->K / kTileK);
   const int nchunks = (nkb + kChunkBlocks - 1) / kChunkBlocks;
   int splits = 1;
