@@ -32,9 +32,8 @@
 //    scales to its block's lanes with one shuffle. 1-bit and 2-bit scales come
 //    with one 8-byte load per lane per four rows (group-of-four scale order).
 //  * Split-K. Slices are spread over CTAs; slice sums go to the workspace and a
-//    small second kernel (programmatic dependent launch, resident beside the main
-//    kernel) adds each row's slice sums in slice order and writes bf16 y: results
-//    are deterministic. (Folding that sum into the main kernel, by the last CTA of a
+//    small second kernel adds each row's slice sums in a fixed order and writes bf16
+//    y: results are deterministic. (Folding that sum into the main kernel, by the last CTA of a
 //    row range or after a meeting of the range's CTAs, measured slower: the tail of
 //    L2 round trips then runs on a handful of SMs.)
 //  * Programmatic dependent launch: before waiting for the previous kernel, each
@@ -319,7 +318,7 @@ __device__ __forceinline__ void build_table(const Args<FMT>& a, int32_t j, uint3
 }
 
 // At most 120 registers a thread (of the SM's 64 K, 61440 for the 512 threads), so
-// that a CTA of the split-K sum kernel (128 threads x 32) fits beside it.
+// that a CTA of the split-K sum kernel (128 threads x 32) always fits beside it.
 template <int FMT>
 __global__ void __maxnreg__(120) gemv_lut_kernel(const Args<FMT> a) {
   using T = Traits<FMT>;
@@ -470,10 +469,9 @@ __global__ void __maxnreg__(120) gemv_lut_kernel(const Args<FMT> a) {
     if (t + i < nt) unit(buf[i], sbuf[i], t + i);
 }
 
-// Sums the slice sums of every row and writes bf16 y. Launched right after the main
-// kernel with programmatic dependent launch: its CTAs become resident while that
-// kernel runs (the main kernel leaves room for one per SM) and wait for its results
-// before reading them. The tail is bound by L2 round trips, so every load of a
+// Sums the slice sums of every row and writes bf16 y, launched right after the main
+// kernel (in plain stream order, see the launch). The tail is bound by L2 round
+// trips, so every load of a
 // thread is issued before its adds: a thread takes a pair of rows (one row when N
 // is odd, where pairs would be misaligned) and a run of at most kSumRun slices; the
 // P threads of a row (consecutive lanes) then combine their runs in a fixed tree
@@ -591,7 +589,13 @@ cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uin
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_lut_kernel<FMT>, a);
   if (e != cudaSuccess || a.KS == 1) return e;
+  // The sum kernel is launched in plain stream order (no programmatic dependent
+  // launch): released early, its CTAs sat waiting beside the main kernel's and came
+  // out of the wait up to 2.5 us apart, which measured slower (the sum's end moved
+  // from ~1.5 to ~4.5 us after the main kernel's). It still lets the next product's
+  // kernel launch early (launch_dependents at its start).
   cudaLaunchConfig_t cfg2 = cfg;
+  cfg2.numAttrs = 0;
   int logP = 0;
   while ((a.KS + (1 << logP) - 1) >> logP > kSumRun) ++logP;
   const bool pairs = (w->N % 2) == 0;
