@@ -35,6 +35,8 @@
 // Every wait is bounded (see sm100_async.cuh).
 #include <cudaTypedefs.h>
 
+#include <utility>
+
 #include "sm100_async.cuh"
 
 namespace {
@@ -93,6 +95,7 @@ struct TcArgs {
   int nacc;         // independent accumulators (a power of two, nacc * tile_m <= 256)
   int kb_per_split; // K blocks per CTA along grid z (split-K)
   float* part;      // [splits][M][N] fp32 partial products, or null (no split)
+  int y_tma;        // 1: Y written through shared memory with one TMA store per tile
   unsigned* fault;
 };
 
@@ -185,6 +188,29 @@ __device__ __forceinline__ uint32_t raw_word(const uint4 (&raw)[7]) {
   return (w & 3) == 0 ? q.x : ((w & 3) == 1 ? q.y : ((w & 3) == 2 ? q.z : q.w));
 }
 
+// Sets word kW (0..27) of a 4-block row chunk held in raw[7].
+template <int kW>
+__device__ __forceinline__ void put_word(uint4 (&raw)[7], uint32_t v) {
+  if constexpr ((kW & 3) == 0) raw[kW >> 2].x = v;
+  else if constexpr ((kW & 3) == 1) raw[kW >> 2].y = v;
+  else if constexpr ((kW & 3) == 2) raw[kW >> 2].z = v;
+  else raw[kW >> 2].w = v;
+}
+// Loads, for the four blocks of a chunk, only the words quarter kQ decodes: quarter
+// 0 reads words 0-1 of a block, 1 words 1-3, 2 words 3-4, 3 words 4-5, and all read
+// word 6 (the scale). Word w of the row is 16 bytes from word w - 1 (group-of-four
+// order) starting at `src`.
+template <int kQ, int kB = 0>
+__device__ __forceinline__ void load_quarter_words(uint4 (&raw)[7], uint32_t src) {
+  constexpr int lo = kQ == 0 ? 0 : (kQ == 1 ? 1 : (kQ == 2 ? 3 : 4));
+  constexpr int hi = kQ == 0 ? 1 : (kQ == 1 ? 3 : (kQ == 2 ? 4 : 5));
+  [&]<int... I>(std::integer_sequence<int, I...>) {
+    ((put_word<7 * kB + lo + I>(raw, lds32(src + 16u * (7 * kB + lo + I)))), ...);
+  }(std::make_integer_sequence<int, hi - lo + 1>{});
+  put_word<7 * kB + 6>(raw, lds32(src + 16u * (7 * kB + 6)));
+  if constexpr (kB < 3) load_quarter_words<kQ, kB + 1>(raw, src);
+}
+
 // Decodes bytes [kJ, kJ1] of block kB into pairs hv[p - kP0] (pairs outside
 // [kP0, kP0 + 16) are skipped). base_e / base_o: the table address of byte 0 for this
 // lane (even / odd entries); V: (s, -s).
@@ -230,7 +256,8 @@ __device__ __forceinline__ void decode_quarter(const uint4 (&raw)[7], int r, uin
 
 __global__ void __launch_bounds__(kThreadsTC, 1)
     gemm_tern_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
-                        const __grid_constant__ CUtensorMap tm_w, const TcArgs a) {
+                        const __grid_constant__ CUtensorMap tm_w,
+                        const __grid_constant__ CUtensorMap tm_y, const TcArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t tab = (sraw + kLowBytes + 0xFFFFu) & ~0xFFFFu;
@@ -261,7 +288,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   load_sel_table(tab, tid);
   if (tid == 0) {
     for (int s = 0; s < kStagesTC; ++s) {
-      mbar_init(fullA + 8 * s, kDecoders);  // every decoder thread arrives
+      mbar_init(fullA + 8 * s, kDecoders / 32);  // every decoder warp arrives
       mbar_init(emptyA + 8 * s, 1);         // the MMA commit arrives
     }
     for (int s = 0; s < kSlabs; ++s) {
@@ -270,7 +297,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
     for (int r = 0; r < kRawStages; ++r) {
       mbar_init(fullR + 8 * r, 1);          // the weight TMA lane arrives (+ bytes)
-      mbar_init(emptyR + 8 * r, kDecoders); // every decoder thread has read its row
+      mbar_init(emptyR + 8 * r, kDecoders / 32); // every decoder warp has read its rows
     }
     mbar_init(accum, 1);
     fence_mbar_init();
@@ -364,11 +391,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     bool ok = true;
     int kb = 0;  // blocks whose store has been issued
     uint32_t hv[16];
-    // the previous block's store has landed: hand its stage to the MMA
+    // the previous block's store has landed: hand its stage to the MMA (one arrival
+    // per warp: 512 single-thread arrivals on one barrier cost about a microsecond)
     auto publish_prev = [&]() {
       tmem_st_wait();
       tc_fence_before_sync();
-      mbar_arrive(fullA + 8 * ((kb - 1) % kStagesTC));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(fullA + 8 * ((kb - 1) % kStagesTC));
     };
     // store block kb once the MMA has released its stage; completes during the next decode
     auto store = [&]() {
@@ -384,15 +413,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     for (int c = 0; c < nchunks; ++c) {
       const int r = c % kRawStages;
       if (ok) ok = mbar_wait(fullR + 8 * r, static_cast<uint32_t>(c / kRawStages) & 1, a.fault, kFaultDecode);
-      uint4 raw[7];
-      // word w of this row: group row >> 2, element 4 w + (row & 3) of the group
+      uint4 raw[7] = {};
+      // word w of this row: group row >> 2, element 4 w + (row & 3) of the group; only
+      // the words this thread's quarter decodes are read (r4 is warp-uniform)
       const uint32_t src = rawring + r * kRawStageBytes +
                            4u * (static_cast<uint32_t>(row >> 2) * kGroupWords + (row & 3));
-#pragma unroll
-      for (int q = 0; q < 7; ++q)
-        raw[q] = make_uint4(lds32(src + 64u * q), lds32(src + 64u * q + 16u),
-                            lds32(src + 64u * q + 32u), lds32(src + 64u * q + 48u));
-      mbar_arrive(emptyR + 8 * r);
+      switch (r4) {
+        case 0: load_quarter_words<0>(raw, src); break;
+        case 1: load_quarter_words<1>(raw, src); break;
+        case 2: load_quarter_words<2>(raw, src); break;
+        default: load_quarter_words<3>(raw, src); break;
+      }
+      __syncwarp();  // the warp's reads of the chunk are done (mbarrier arrive releases them)
+      if (lane == 0) mbar_arrive(emptyR + 8 * r);
       decode_quarter<0>(raw, r4, base_e, base_o, hv);
       if (kb > 0) publish_prev();
       store();
@@ -423,28 +456,66 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
     // every accumulator received at least one MMA: K >= 128 gives 8 per block
     const int nacc_used = a.nacc < 8 * nkb ? a.nacc : 8 * nkb;
-    for (int c0 = 16 * grp; c0 < a.tile_m; c0 += 64) {
-      uint32_t v[16];
-      tmem_ld16(lane_base + static_cast<uint32_t>(c0), v);
-      tmem_ld_wait();
-      for (int j = 1; j < nacc_used; ++j) {  // accumulators summed in order
-        uint32_t u[16];
-        tmem_ld16(lane_base + static_cast<uint32_t>(j * a.tile_m + c0), u);
+    if (a.y_tma) {
+      // bf16 tile [tokens][128 rows] staged in shared memory (the activation slabs are
+      // free once the accumulator is complete), then one TMA store; the tokens'
+      // exponents first go to shared memory (below the table, where slab 0 was)
+      const uint32_t ot = tab + kHighB;
+      int* xe = reinterpret_cast<int*>(smem_raw + (bstage0 - sraw));
+      for (int t = tid - 128; t < a.tile_m; t += kDecoders)
+        xe[t] = m0 + t < a.M ? a.xexp[m0 + t] : 0;
+      named_bar_sync(3, kDecoders);
+      const int rloc = 32 * q + lane;
+      for (int c0 = 16 * grp; c0 < a.tile_m; c0 += 64) {
+        uint32_t v[16];
+        tmem_ld16(lane_base + static_cast<uint32_t>(c0), v);
         tmem_ld_wait();
+        for (int j = 1; j < nacc_used; ++j) {  // accumulators summed in order
+          uint32_t u[16];
+          tmem_ld16(lane_base + static_cast<uint32_t>(j * a.tile_m + c0), u);
+          tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(u[i]));
-      }
-      if (!ok || ne >= a.N) continue;
+          for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(u[i]));
+        }
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int64_t m = m0 + c0 + i;
-        if (m < a.M) {
+        for (int i = 0; i < 16; ++i) {
           // undo the activation row's power-of-two scaling (exact)
-          const float y = ldexpf(__uint_as_float(v[i]), a.xexp[m]);
-          if (a.part)
-            a.part[(static_cast<int64_t>(blockIdx.z) * a.M + m) * a.N + ne] = y;
-          else
-            a.Y[m * a.N + ne] = f32_to_bf16_bits(y);
+          const float y = ldexpf(__uint_as_float(v[i]), xe[c0 + i]);
+          const uint32_t addr = ot + static_cast<uint32_t>((c0 + i) * 256 + rloc * 2);
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(f32_to_bf16_bits(y)) : "memory");
+        }
+      }
+      fence_proxy_async_smem();  // the generic-proxy writes, before the TMA reads them
+      named_bar_sync(3, kDecoders);
+      if (tid == 128 && ok) {
+        tma_store_2d(&tm_y, ot, static_cast<int32_t>(n0), static_cast<int32_t>(m0));
+        bulk_commit_group();
+        bulk_wait_group_read0();
+      }
+    } else {
+      for (int c0 = 16 * grp; c0 < a.tile_m; c0 += 64) {
+        uint32_t v[16];
+        tmem_ld16(lane_base + static_cast<uint32_t>(c0), v);
+        tmem_ld_wait();
+        for (int j = 1; j < nacc_used; ++j) {  // accumulators summed in order
+          uint32_t u[16];
+          tmem_ld16(lane_base + static_cast<uint32_t>(j * a.tile_m + c0), u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(u[i]));
+        }
+        if (!ok || ne >= a.N) continue;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int64_t m = m0 + c0 + i;
+          if (m < a.M) {
+            // undo the activation row's power-of-two scaling (exact)
+            const float y = ldexpf(__uint_as_float(v[i]), a.xexp[m]);
+            if (a.part)
+              a.part[(static_cast<int64_t>(blockIdx.z) * a.M + m) * a.N + ne] = y;
+            else
+              a.Y[m * a.N + ne] = f32_to_bf16_bits(y);
+          }
         }
       }
     }
@@ -612,9 +683,23 @@ cudaError_t lbq_launch_gemm_tc(const lbq_weights* w, const uint16_t* X, int64_t 
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  // Y through shared memory and one TMA store per tile when the tensor map can
+  // describe it (16-byte aligned base and row pitch) and K is not split
+  CUtensorMap ty;
+  a.y_tma = 0;
+  if (!a.part && (reinterpret_cast<uintptr_t>(Y) & 15) == 0 && (w->N * 2) % 16 == 0) {
+    const cuuint64_t ydims[2] = {static_cast<cuuint64_t>(w->N), static_cast<cuuint64_t>(M)};
+    const cuuint64_t ystrides[1] = {static_cast<cuuint64_t>(w->N) * 2};
+    const cuuint32_t ybox[2] = {static_cast<cuuint32_t>(kTileN), static_cast<cuuint32_t>(a.tile_m)};
+    if (fn(&ty, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, Y, ydims, ystrides, ybox, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+      a.y_tma = 1;
+  }
+  if (!a.y_tma) ty = tw;  // unused
   dim3 grid(static_cast<unsigned>((w->N + kTileN - 1) / kTileN),
             static_cast<unsigned>((M + a.tile_m - 1) / a.tile_m), static_cast<unsigned>(plan.splits));
-  gemm_tern_tc_kernel<<<grid, kThreadsTC, kSmemTC, s>>>(tm, tw, a);
+  gemm_tern_tc_kernel<<<grid, kThreadsTC, kSmemTC, s>>>(tm, tw, ty, a);
   e = cudaGetLastError();
   if (e != cudaSuccess || plan.splits == 1) return e;
   const int64_t MN = M * w->N;
