@@ -578,13 +578,26 @@ struct TcPlan {
 // cannot fill the SMs (small batches).
 TcPlan plan_for(const lbq_weights* w, int64_t M) {
   TcPlan p;
-  // 256 tokens per tile (the widest MMA, which also hides an MMA's latency behind the
-  // next) unless that leaves SMs idle, then 128; small batches round up to 16.
   const int64_t ntiles = (w->N + kTileN - 1) / kTileN;
-  if (M >= 256 && ntiles * ((M + 255) / 256) >= sm_count())
-    p.tile_m = 256;
-  else
-    p.tile_m = M >= 128 ? 128 : static_cast<int>((M + 15) / 16 * 16);
+  if (M >= 128 && ntiles * ((M + kMaxTileM - 1) / kMaxTileM) >= 3 * sm_count()) {
+    p.tile_m = kMaxTileM;  // many waves of full-width tiles: the tail matters little
+  } else if (M >= 128) {
+    // Few waves: choose the token tile (a multiple of 16, 128..256) that minimises the
+    // modelled time: waves of CTAs x (the tile's MMA time, which stops shrinking below
+    // ~160 tokens because an MMA then waits on the previous one, + a fixed cost per tile).
+    int64_t best = -1;
+    for (int t = 128; t <= kMaxTileM; t += 16) {
+      const int64_t tiles = ntiles * ((M + t - 1) / t);
+      const int64_t waves = (tiles + sm_count() - 1) / sm_count();
+      const int64_t cost = waves * ((t > 160 ? t : 160) + 32);
+      if (best < 0 || cost < best || (cost == best && t > p.tile_m)) {
+        best = cost;
+        p.tile_m = t;
+      }
+    }
+  } else {
+    p.tile_m = static_cast<int>((M + 15) / 16 * 16);
+  }
   const int64_t tiles = ntiles * ((M + p.tile_m - 1) / p.tile_m);
   const int nkb = static_cast<int>(w->K / kTileK);
   const int nchunks = (nkb + kChunkBlocks - 1) / kChunkBlocks;
