@@ -611,18 +611,6 @@ TcPlan plan_for(const lbq_weights* w, int64_t M) {
   return p;
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn_tc() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace
@@ -673,7 +661,7 @@ cudaError_t lbq_launch_gemm_tc(const lbq_weights* w, const uint16_t* X, int64_t 
   a.fault = lbq_fault_word();
   if (!a.fault) return cudaErrorInvalidDevicePointer;
 
-  auto fn = encode_fn_tc();
+  auto fn = tensor_map_encoder();
   if (!fn) return cudaErrorInvalidValue;
   CUtensorMap tm;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(w->K), static_cast<cuuint64_t>(M)};

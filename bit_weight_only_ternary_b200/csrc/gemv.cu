@@ -17,11 +17,13 @@
 //    handles the same word position of a row, and the table is laid out
 //    [value][lane], so table reads never collide on a bank.
 //  * Streaming. The packed rows are stored in groups of four (word w of four rows
-//    in 16 consecutive bytes), so one coalesced 16-byte load per lane brings a
-//    lane its word of four rows: a warp load covers 448 (ternary) or 512 bytes.
-//    Loads go straight to registers, three 16-row units in flight per warp; no
-//    shared-memory staging, whose extra write and read would cost shared-memory
-//    bandwidth, the kernel's second bound.
+//    in 16 consecutive bytes), so a 16-row unit's slice is four runs of 448
+//    (ternary) or 512 bytes. One warp issues tensor copies (TMA) of four units at
+//    a time (7 to 10 KB) into a ring of shared-memory slots; the 16 compute warps
+//    take one unit each and read their lane's word of four rows with one 16-byte
+//    shared load per group. (Per-unit copies, 1.8 KB each, streamed at half the
+//    rate: the copy engine keeps few copies in flight. Loads into registers
+//    instead queue in the L1 path ahead of the x slice and the table build.)
 //  * Reduction. Each lane holds one word's partial sum for each of 16 rows; a
 //    transpose-reduce butterfly (16 shuffles) leaves row l's slice sum in lane l.
 //    (Rotating the group order per lane would spare the selects of two stages, but
@@ -36,12 +38,11 @@
 //    y: results are deterministic. (Folding that sum into the main kernel, by the last CTA of a
 //    row range or after a meeting of the range's CTAs, measured slower: the tail of
 //    L2 round trips then runs on a handful of SMs.)
-//  * Programmatic dependent launch: before waiting for the previous kernel, each
-//    warp asks L2 to prefetch its first units of weights (a hint only: the loads
-//    that feed the arithmetic are issued after the wait, so weights written by the
-//    previous kernel are always read correctly).
-#include <cudaTypedefs.h>
-
+//  * Programmatic dependent launch: the copy warp never waits for the previous
+//    kernel, so the ring fills while it finishes. Only the batch-1 kernels let
+//    their successor start early, and they never write packed weights; any other
+//    kernel has completed before this one starts. x, y and the workspace are
+//    touched only after the wait.
 #include <type_traits>
 
 #include "rht.cuh"
@@ -51,32 +52,49 @@ namespace {
 
 using namespace lbq;
 
-constexpr int kWarps = 16;
-constexpr int kThreads = 32 * kWarps;
-constexpr int kRows = 16;           // rows per unit (four groups of four)
-constexpr int kAhead = 3;           // units in flight per warp
-constexpr uint32_t kPage = 65536;   // table page: 256 values x 256 bytes
+constexpr int kWarps = 16;                    // consumer warps
+constexpr int kThreads = 32 * kWarps;         // consumer threads
+constexpr int kBlockThreads = kThreads + 32;  // + the copy-issuing warp
+constexpr int kRows = 16;                     // rows per unit (four groups of four)
+constexpr int kSub = 4;                       // units per ring slot (one tensor copy)
+constexpr uint32_t kPage = 65536;             // table page: 256 values x 256 bytes
 // Shared memory: the 128 KB table at the first 64 KB boundary of the window (its
-// page addressing keeps the base in the upper half of the PRMT operand), the x
-// slice below it. The dynamic window starts 1 KB into shared memory on sm_100, so
-// [1 KB, 64 KB) holds the x slice; a window starting at 0 puts x above the table.
-constexpr uint32_t kXBytes = 4096;  // up to 1024 fp32
-constexpr uint32_t kSmem = (kPage - 1024) + 2 * kPage + kXBytes;
-constexpr unsigned kFaultLayout = 3;
+// page addressing keeps the base in the upper half of the PRMT operand); below it
+// (the dynamic window starts 1 KB into shared memory on sm_100) the x slice, the
+// mbarriers and the first ring slots, above it the other ring slots. A window that
+// starts at 0 puts everything above the table.
+constexpr uint32_t kXBytes = 4096;  // the slice of x as fp32 (up to 1024)
+constexpr int kMaxSlots = 32;
+// x and the mbarriers, rounded up so that the ring slots after them stay 128-byte
+// aligned, as tensor copies into shared memory require
+constexpr uint32_t kMisc = (kXBytes + 2 * 8 * kMaxSlots + 1023) & ~1023u;
+// 225 KB: with the 1 KB every CTA reserves, a CTA of the split-K sum kernel still
+// fits beside this one in the SM's 228 KB.
+constexpr uint32_t kSmem = 225 * 1024;
+constexpr unsigned kFaultLayout = 3, kFaultRing = 10;
 
 template <int FMT>
 struct Traits;
+// kGroupBytes: a group of four rows' codes in one slice; kScaleBytes: its scales
+// (1-bit and 2-bit; ternary scales sit among the codes); kSlot: a ring slot of kSub
+// 16-row units, codes first, then scales.
 template <>
 struct Traits<LBQ_TERN5> {
   static constexpr int kWeights = 512, kWords = 28, kBlocks = 4, kDigits = 5;
+  static constexpr uint32_t kGroupBytes = 16 * kWords, kScaleBytes = 0;
+  static constexpr uint32_t kSlot = 4 * kSub * (kGroupBytes + kScaleBytes);
 };
 template <>
 struct Traits<LBQ_SIGN1> {
   static constexpr int kWeights = 1024, kWords = 32, kBlocks = 8, kDigits = 8;
+  static constexpr uint32_t kGroupBytes = 16 * kWords, kScaleBytes = 8 * kBlocks;
+  static constexpr uint32_t kSlot = 4 * kSub * (kGroupBytes + kScaleBytes);
 };
 template <>
 struct Traits<LBQ_Q2RHT> {
   static constexpr int kWeights = 512, kWords = 32, kBlocks = 16, kDigits = 4;
+  static constexpr uint32_t kGroupBytes = 16 * kWords, kScaleBytes = 8 * kBlocks;
+  static constexpr uint32_t kSlot = 4 * kSub * (kGroupBytes + kScaleBytes);
 };
 
 // Word of the slice that lane l handles (ternary: block l/8, word l%8 of it; lanes
@@ -132,18 +150,16 @@ __device__ __forceinline__ float lds_imm(uint32_t addr) {
   asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(kImm));
   return v;
 }
-__device__ __forceinline__ uint4 ldg_stream16(const void* p) {
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
   uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.b32 {%0, %1, %2, %3}, [%4];"
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
+               : "r"(addr));
   return v;
 }
-__device__ __forceinline__ uint2 ldg_stream8(const void* p) {
+__device__ __forceinline__ uint2 lds_v2(uint32_t addr) {
   uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.b32 {%0, %1}, [%2];"
-               : "=r"(v.x), "=r"(v.y)
-               : "l"(p));
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
 }
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
@@ -167,9 +183,9 @@ __device__ __forceinline__ float2 lookup_pair(uint32_t w0, uint32_t w1, uint32_t
   return __fadd2_rn(__fadd2_rn(e0, e1), __fadd2_rn(e2, e3));
 }
 
-// The x slice of slice j, in flight: the loads are issued by x_issue (before the
-// weight loads, so that the table build, which waits for x, is not queued behind
-// them) and stored to shared memory as fp32 by x_store.
+// The x slice of slice j, loaded by x_issue (plain loads: the weights come through
+// the copy engine, whose queue would hold x back behind them) and stored to shared
+// memory as fp32 by x_store.
 struct XLoad {
   uint4 v0, v1, d;
 };
@@ -314,81 +330,120 @@ __device__ __forceinline__ void build_table(const Args<FMT>& a, int32_t j, uint3
       }
     }
   }
-  __syncthreads();
+  named_bar_sync(1, kThreads);
 }
 
-// At most 120 registers a thread (of the SM's 64 K, 61440 for the 512 threads), so
-// that a CTA of the split-K sum kernel (128 threads x 32) always fits beside it.
+// One CTA: kWarps consumer warps and one warp that issues the weight copies. At most
+// 112 registers a thread (544 x 112 = 60928 of the SM's 65536), so that a CTA of the
+// split-K sum kernel (128 threads x 32) always fits beside it. tm_c / tm_s: the
+// codes / scales as tensor maps with a box of kSub units (tm_c1 / tm_s1: one unit).
 template <int FMT>
-__global__ void __maxnreg__(120) gemv_lut_kernel(const Args<FMT> a) {
+__global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtensorMap tm_c,
+                                                 const __grid_constant__ CUtensorMap tm_s,
+                                                 const __grid_constant__ CUtensorMap tm_c1,
+                                                 const __grid_constant__ CUtensorMap tm_s1,
+                                                 const Args<FMT> a) {
   using T = Traits<FMT>;
   constexpr bool kSepScales = FMT != LBQ_TERN5;
+  constexpr uint32_t kScaleOff = 4 * kSub * T::kGroupBytes;  // scales within a slot
+  static_assert(T::kSlot % 128 == 0 && kScaleOff % 128 == 0 && (4 * T::kGroupBytes) % 128 == 0 &&
+                    (4 * T::kScaleBytes) % 128 == 0,
+                "tensor copies land on 128-byte boundaries");
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_launch_dependents();
 
+  // ---- shared-memory layout (see the constants)
   const uint32_t sbase = smem_u32(smem);
+  const uint32_t send = sbase + kSmem;
   const uint32_t tbase = (sbase + kPage - 1) & ~(kPage - 1);
-  const uint32_t xaddr = (tbase - sbase >= kXBytes) ? sbase : tbase + 2 * kPage;
-  if (tbase + 2 * kPage > sbase + kSmem || xaddr + kXBytes > sbase + kSmem) {
+  const uint32_t ttop = tbase + 2 * kPage;
+  const bool misc_low = tbase - sbase >= kMisc;
+  const uint32_t misc = misc_low ? sbase : ttop;
+  const uint32_t lo0 = misc_low ? sbase + kMisc : sbase;  // ring slots below the table
+  const uint32_t hi0 = misc_low ? ttop : ttop + kMisc;    // ... and above it
+  const int s_lo = static_cast<int>((tbase - lo0) / T::kSlot);
+  const int s_hi = hi0 < send ? static_cast<int>((send - hi0) / T::kSlot) : 0;
+  const int S = s_lo + s_hi < kMaxSlots ? s_lo + s_hi : kMaxSlots;
+  if (ttop > send || misc + kMisc > send || S < kWarps / kSub + 2 || ((lo0 | hi0) & 127) != 0) {
     if (tid == 0) atomicExch(a.fault, kFaultLayout);  // cannot happen with a 0 or 1 KB prefix
     return;
   }
-  float* xs = reinterpret_cast<float*>(smem + (xaddr - sbase));
+  float* xs = reinterpret_cast<float*>(smem + (misc - sbase));
+  const uint32_t full0 = misc + kXBytes, empty0 = full0 + 8 * kMaxSlots;
+  auto slot_addr = [&](int s) {
+    return s < s_lo ? lo0 + static_cast<uint32_t>(s) * T::kSlot
+                    : hi0 + static_cast<uint32_t>(s - s_lo) * T::kSlot;
+  };
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, kSub);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
 
   // This CTA: slice j, units [u_lo, u_hi) of kRows rows (a.G CTAs share a slice).
   // 32-bit arithmetic: NU <= 2^15 and G <= the SM count.
   const int32_t NU = static_cast<int32_t>((a.N + kRows - 1) / kRows);
-  const int32_t NG = static_cast<int32_t>((a.N + 3) / 4);  // groups of four rows present
   const int32_t j = static_cast<int32_t>(blockIdx.x) / a.G;
   const int32_t gs = static_cast<int32_t>(blockIdx.x) - j * a.G;
   const int32_t u_lo = static_cast<int32_t>(static_cast<uint32_t>(gs * NU) / static_cast<uint32_t>(a.G));
   const int32_t u_hi =
       static_cast<int32_t>(static_cast<uint32_t>((gs + 1) * NU) / static_cast<uint32_t>(a.G));
   const int32_t n_units = u_hi - u_lo;
-
   const int blk0 = j * T::kBlocks;
   const int nb = a.nblk - blk0 < T::kBlocks ? a.nblk - blk0 : T::kBlocks;
-  const int wl = lane_word<FMT>(lane, nb);
-  const int64_t gstride = 4 * a.cstride;  // bytes per group of four rows
-  const uint8_t* slice = a.codes + static_cast<int64_t>(16) * j * T::kWords;
-  // Lanes without a word (their table columns are zero) read word 0 of the slice:
-  // every load is in bounds and none needs a predicate.
-  const uint8_t* cptr = slice + 16 * (wl < 0 ? 0 : wl);
-  // 1-bit / 2-bit: this lane's block scales of four rows are 8 bytes of the group
-  // (a lane without a word reads the slice's first block: finite, times zero).
-  const int sblk = wl < 0 ? blk0 : blk0 + (FMT == LBQ_SIGN1 ? (lane >> 2) : (lane >> 1));
-  const uint16_t* sptr = kSepScales ? a.scales + 4 * sblk : nullptr;
-  const int64_t sgstride = 4 * a.sstride;
 
-  // Ask L2 for this warp's first units (a hint; the real loads follow the wait).
-  if (lane < 4 * kAhead) {
-    const int32_t u = u_lo + warp + kWarps * (lane >> 2);
-    const int32_t g = 4 * u + (lane & 3);
-    const int64_t words_left = a.cstride / 4 - static_cast<int64_t>(j) * T::kWords;
-    const uint32_t bytes = 16u * static_cast<uint32_t>(words_left < T::kWords ? words_left : T::kWords);
-    if (u < u_hi && g < NG) prefetch_l2_bulk(slice + g * gstride, bytes);
+  if (warp == kWarps) {
+    // ---- copies: slot sequence number q holds units kSub q .. kSub q + kSub - 1 of
+    // this CTA and goes to slot q % S; one tensor copy of their groups' slice (groups
+    // past the last read as zero) and one of their scales; a last, partial slot gets
+    // one copy per unit. The packed weights are never written by a kernel that lets
+    // this one start early (only the batch-1 kernels do, and they do not write
+    // weights), so the copies do not wait for the previous kernel: the ring fills
+    // while it finishes.
+    if (lane == 0) {
+      prefetch_tmap(&tm_c);
+      prefetch_tmap(&tm_c1);
+      if (kSepScales) {
+        prefetch_tmap(&tm_s);
+        prefetch_tmap(&tm_s1);
+      }
+      const int32_t cx = j * 4 * T::kWords, sx = 4 * blk0;
+      const int32_t nslots = (n_units + kSub - 1) / kSub;
+      int slot = 0;
+      uint32_t round = 0;
+      for (int32_t q = 0; q < nslots; ++q) {
+        const uint32_t full = full0 + 8 * slot;
+        if (round > 0 && !mbar_wait(empty0 + 8 * slot, (round - 1) & 1, a.fault, kFaultRing)) break;
+        const uint32_t dst = slot_addr(slot);
+        const int32_t u0 = kSub * q;
+        const int32_t nu = n_units - u0 < kSub ? n_units - u0 : kSub;
+        const int32_t g0 = 4 * (u_lo + u0);
+        mbar_arrive_expect_tx(full, static_cast<uint32_t>(nu) * 4 * (T::kGroupBytes + T::kScaleBytes));
+        if (nu == kSub) {
+          tma_load_2d(dst, &tm_c, cx, g0, full);
+          if (kSepScales) tma_load_2d(dst + kScaleOff, &tm_s, sx, g0, full);
+        } else {
+          for (int32_t i = 0; i < nu; ++i) {
+            tma_load_2d(dst + i * 4 * T::kGroupBytes, &tm_c1, cx, g0 + 4 * i, full);
+            if (kSepScales)
+              tma_load_2d(dst + kScaleOff + i * 4 * T::kScaleBytes, &tm_s1, sx, g0 + 4 * i, full);
+          }
+        }
+        if (++slot == S) {
+          slot = 0;
+          ++round;
+        }
+      }
+    }
+    return;  // the consumers synchronise among themselves from here on
   }
 
-  uint4 buf[kAhead][4];
-  uint2 sbuf[kAhead][4];
-  // This warp's units: u_lo + warp + kWarps t for t < nt. Groups past the last row
-  // (the matrix's last unit) reload the last group: those rows are never written.
-  const int32_t nt = n_units > warp ? (n_units - warp + kWarps - 1) / kWarps : 0;
-  const uint32_t gstride32 = static_cast<uint32_t>(gstride);
-  const uint32_t sgstride32 = static_cast<uint32_t>(sgstride);
-  auto load = [&](uint4 (&b)[4], uint2 (&sb)[4], int32_t t) {
-    const uint32_t g0 = 4u * static_cast<uint32_t>(u_lo + warp + kWarps * t);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t g = min(g0 + q, static_cast<uint32_t>(NG - 1));
-      b[q] = ldg_stream16(cptr + static_cast<uint64_t>(g) * gstride32);
-      if (kSepScales) sb[q] = ldg_stream8(sptr + static_cast<uint64_t>(g) * sgstride32);
-    }
-  };
-
-  // ... and for the x slice (written by the previous kernel in a chain of products:
-  // a prefetch into L2 is only a hint and cannot return stale data)
+  // ... and the x slice, which the previous kernel of a chain of products may write:
+  // a prefetch into L2 is only a hint and cannot return stale data
   if (tid >= 480 && tid - 480 < T::kWeights / 64) {
     const int64_t k = static_cast<int64_t>(j) * T::kWeights + 64 * (tid - 480);
     if (k + 64 <= a.K) prefetch_l2_bulk(a.x + k, 128);
@@ -397,16 +452,17 @@ __global__ void __maxnreg__(120) gemv_lut_kernel(const Args<FMT> a) {
   }
 
   pdl_wait();  // x, y and the workspace may belong to the previous kernel until here
-  // x first, alone, then the table: weight loads issued beside them would queue
-  // ahead of them (the first units' weights were prefetched into L2 above)
   x_store<FMT>(x_issue<FMT>(a, j, tid), xs, tid);
-  __syncthreads();
-  if (nt > 0) load(buf[0], sbuf[0], 0);  // one unit in flight during the build
+  named_bar_sync(1, kThreads);
   build_table<FMT>(a, j, tbase, xs, tid);
-#pragma unroll
-  for (int i = 1; i < kAhead; ++i)
-    if (i < nt) load(buf[i], sbuf[i], i);
 
+  // This lane's word of each group, and (1-bit, 2-bit) its block's scales of four
+  // rows: lanes without a word (their table columns are zero) read word 0 and the
+  // slice's first block.
+  const int wl = lane_word<FMT>(lane, nb);
+  const uint32_t woff = 16u * static_cast<uint32_t>(wl < 0 ? 0 : wl);
+  const int sblk = wl < 0 ? 0 : (FMT == LBQ_SIGN1 ? (lane >> 2) : (lane >> 1));
+  const uint32_t soff = kScaleOff + 8u * static_cast<uint32_t>(sblk);
   const uint32_t lanereg = tbase | static_cast<uint32_t>(lane * 4);
   const int src6 = (lane & ~7) | 6;  // ternary: the lane holding this block's scale word
   const int64_t NR = a.N;
@@ -456,17 +512,36 @@ __global__ void __maxnreg__(120) gemv_lut_kernel(const Args<FMT> a) {
         part_j[row] = acc[0];
     }
   };
-  int32_t t = 0;
-  for (; t + kAhead <= nt; t += kAhead) {
+  // ---- consumers: warp w takes units w, w + kWarps, ...; unit tg sits in slot
+  // sequence number tg / kSub at place tg % kSub (= w % kSub)
+  const uint32_t sub = static_cast<uint32_t>(warp % kSub);
+  const int32_t nt = n_units > warp ? (n_units - warp + kWarps - 1) / kWarps : 0;
+  int slot = warp / kSub;
+  uint32_t round = 0;
+  for (int32_t t = 0; t < nt; ++t) {
+    if (!mbar_wait(full0 + 8 * slot, round & 1, a.fault, kFaultRing)) break;
+    const uint32_t src = slot_addr(slot);
+    uint4 b[4];
+    uint2 sb[4];
 #pragma unroll
-    for (int i = 0; i < kAhead; ++i) {
-      unit(buf[i], sbuf[i], t + i);
-      if (t + i + kAhead < nt) load(buf[i], sbuf[i], t + i + kAhead);
+    for (int q = 0; q < 4; ++q) {
+      b[q] = lds_v4(src + (4 * sub + q) * T::kGroupBytes + woff);
+      sb[q] = kSepScales ? lds_v2(src + soff + (4 * sub + q) * T::kScaleBytes) : make_uint2(0u, 0u);
+    }
+    unit(b, sb, t);
+    // The warp has used its words: the slot goes back to the copies (the warp barrier
+    // and the proxy fence order these reads before the copy engine's next writes).
+    __syncwarp();
+    if (lane == 0) {
+      fence_proxy_async_smem();
+      mbar_arrive(empty0 + 8 * slot);
+    }
+    slot += kWarps / kSub;
+    if (slot >= S) {
+      slot -= S;
+      ++round;
     }
   }
-#pragma unroll
-  for (int i = 0; i < kAhead - 1; ++i)
-    if (t + i < nt) unit(buf[i], sbuf[i], t + i);
 }
 
 // Sums the slice sums of every row and writes bf16 y, launched right after the main
@@ -579,7 +654,7 @@ cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uin
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kBlockThreads);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -587,7 +662,39 @@ cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uin
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_lut_kernel<FMT>, a);
+  // The packed weights as tensor maps for the ring's copies: codes as 32-bit words,
+  // one row of the map per group of four rows; 1-bit / 2-bit scales as fp16, one row
+  // per group. Boxes cover one slice of kSub units (and of one unit, for the tail).
+  using T = Traits<FMT>;
+  auto fn = tensor_map_encoder();
+  if (!fn) return cudaErrorInvalidValue;
+  const cuuint64_t NG = static_cast<cuuint64_t>((w->N + 3) / 4);
+  auto encode = [&](CUtensorMap* m, CUtensorMapDataType dt, void* base, cuuint64_t cols,
+                    cuuint64_t pitch, cuuint32_t bx, cuuint32_t by) {
+    const cuuint64_t dims[2] = {cols, NG};
+    const cuuint64_t strides[1] = {pitch};
+    const cuuint32_t box[2] = {bx, by};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
+  CUtensorMap tm_c, tm_c1, tm_s, tm_s1;
+  void* codes = const_cast<void*>(w->codes);
+  const cuuint64_t cw = static_cast<cuuint64_t>(w->code_stride);  // words per group
+  if (!encode(&tm_c, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, cw, cw * 4, 4 * T::kWords, 4 * kSub) ||
+      !encode(&tm_c1, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, cw, cw * 4, 4 * T::kWords, 4))
+    return cudaErrorInvalidValue;
+  tm_s = tm_c;  // ternary: unused
+  tm_s1 = tm_c1;
+  if (T::kScaleBytes > 0) {
+    void* sc = const_cast<void*>(w->scales);
+    const cuuint64_t se = static_cast<cuuint64_t>(w->scale_stride) * 4;  // fp16 per group
+    if (!encode(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, sc, se, se * 2, T::kScaleBytes / 2, 4 * kSub) ||
+        !encode(&tm_s1, CU_TENSOR_MAP_DATA_TYPE_UINT16, sc, se, se * 2, T::kScaleBytes / 2, 4))
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_lut_kernel<FMT>, tm_c, tm_s, tm_c1, tm_s1, a);
   if (e != cudaSuccess || a.KS == 1) return e;
   // The sum kernel is launched in plain stream order (no programmatic dependent
   // launch): released early, its CTAs sat waiting beside the main kernel's and came
@@ -601,7 +708,9 @@ cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uin
   const bool pairs = (w->N % 2) == 0;
   const int64_t threads = (pairs ? w->N / 2 : w->N) << logP;
   const int64_t ctas = (threads + kSumThreads - 1) / kSumThreads;
-  cfg2.gridDim = dim3(static_cast<unsigned>(ctas < sm_count() ? ctas : sm_count()));
+  // one pass per thread: up to two of its 4096-register CTAs an SM once the main
+  // kernel has left (the next product's main kernel waits for the space)
+  cfg2.gridDim = dim3(static_cast<unsigned>(ctas < 8 * sm_count() ? ctas : 8 * sm_count()));
   cfg2.blockDim = dim3(kSumThreads);
   cfg2.dynamicSmemBytes = 0;
   const float* part = a.part;

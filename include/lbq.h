@@ -193,7 +193,8 @@ lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const in
  * current device since the last query, and clears that record. Every wait in the
  * kernels (on an mbarrier, for a TMA copy or a slot) is bounded by about 2 s; a
  * wait that runs out records a non-zero *code (3: shared-memory layout of the
- * batch-1 product, 4-9: tensor-core product stages) and the kernel returns early
+ * batch-1 product, 4-9: tensor-core product stages, 10: the batch-1 product's
+ * weight copies) and the kernel returns early
  * with incomplete outputs instead of hanging. A non-zero code means a library fault. Synchronises the device.
  * Errors: LBQ_ERR_ARG (code NULL), LBQ_ERR_CUDA. */
 lbq_status lbq_device_fault(uint32_t* code);
