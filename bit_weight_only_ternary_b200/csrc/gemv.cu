@@ -346,6 +346,7 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
   using T = Traits<FMT>;
   constexpr bool kSepScales = FMT != LBQ_TERN5;
   constexpr uint32_t kScaleOff = 4 * kSub * T::kGroupBytes;  // scales within a slot
+  static_assert(kWarps % kSub == 0, "whole warp groups");
   static_assert(T::kSlot % 128 == 0 && kScaleOff % 128 == 0 && (4 * T::kGroupBytes) % 128 == 0 &&
                     (4 * T::kScaleBytes) % 128 == 0,
                 "tensor copies land on 128-byte boundaries");
@@ -364,8 +365,13 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
   const uint32_t hi0 = misc_low ? ttop : ttop + kMisc;    // ... and above it
   const int s_lo = static_cast<int>((tbase - lo0) / T::kSlot);
   const int s_hi = hi0 < send ? static_cast<int>((send - hi0) / T::kSlot) : 0;
-  const int S = s_lo + s_hi < kMaxSlots ? s_lo + s_hi : kMaxSlots;
-  if (ttop > send || misc + kMisc > send || S < kWarps / kSub + 2 || ((lo0 | hi0) & 127) != 0) {
+  // The slot count is a multiple of the kWarps / kSub warp groups: unit sequence
+  // number q goes to slot q % S and is taken by group q % (kWarps / kSub), so every
+  // slot belongs to one group, which waits for a slot's next fill only after taking
+  // the previous one (an mbarrier parity wait never looks two phases ahead).
+  constexpr int kGroups = kWarps / kSub;
+  const int S = (s_lo + s_hi < kMaxSlots ? s_lo + s_hi : kMaxSlots) / kGroups * kGroups;
+  if (ttop > send || misc + kMisc > send || S < 2 * kGroups || ((lo0 | hi0) & 127) != 0) {
     if (tid == 0) atomicExch(a.fault, kFaultLayout);  // cannot happen with a 0 or 1 KB prefix
     return;
   }
@@ -536,7 +542,7 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
       fence_proxy_async_smem();
       mbar_arrive(empty0 + 8 * slot);
     }
-    slot += kWarps / kSub;
+    slot += kGroups;
     if (slot >= S) {
       slot -= S;
       ++round;
