@@ -352,7 +352,6 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
                 "tensor copies land on 128-byte boundaries");
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  pdl_launch_dependents();
 
   // ---- shared-memory layout (see the constants)
   const uint32_t sbase = smem_u32(smem);
@@ -548,6 +547,9 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
       ++round;
     }
   }
+  // The split-K sum kernel may start once every CTA is past its units (the copy warp
+  // has left already): its CTAs then sit beside the last ones for a short wait only.
+  pdl_launch_dependents();
 }
 
 // Sums the slice sums of every row and writes bf16 y, launched right after the main
@@ -702,13 +704,11 @@ cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uin
   }
   cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_lut_kernel<FMT>, tm_c, tm_s, tm_c1, tm_s1, a);
   if (e != cudaSuccess || a.KS == 1) return e;
-  // The sum kernel is launched in plain stream order (no programmatic dependent
-  // launch): released early, its CTAs sat waiting beside the main kernel's and came
-  // out of the wait up to 2.5 us apart, which measured slower (the sum's end moved
-  // from ~1.5 to ~4.5 us after the main kernel's). It still lets the next product's
-  // kernel launch early (launch_dependents at its start).
+  // The sum kernel is launched early too (the main kernel lets it start when its
+  // CTAs are past their units; released at the main kernel's start instead, its CTAs
+  // came out of the wait up to 3 us apart). It lets the next product's kernel
+  // launch early in turn (launch_dependents at its start).
   cudaLaunchConfig_t cfg2 = cfg;
-  cfg2.numAttrs = 0;
   int logP = 0;
   while ((a.KS + (1 << logP) - 1) >> logP > kSumRun) ++logP;
   const bool pairs = (w->N % 2) == 0;
