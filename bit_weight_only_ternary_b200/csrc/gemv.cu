@@ -275,17 +275,17 @@ __device__ __forceinline__ void build_table(const Args<FMT>& a, int32_t j, uint3
       const float l0f = static_cast<float>(m % 3 - 1), l1f = static_cast<float>(m / 3 - 1);
       ab[m] = __ffma2_rn(make_float2(l0f, l0f), xv[0], __fmul2_rn(make_float2(l1f, l1f), xv[1]));
     }
-    for (int hi = tid >> 6; hi < 9; hi += kStep) {
+    // 27 runs of 9 values (digits 2..4 fixed) per column pair, dealt round-robin:
+    // at most 4 runs a thread
+    for (int hd = tid >> 6; hd < 27; hd += kStep) {
+      const int hi = hd / 3, d2 = hd - 3 * hi;
       const float l3 = static_cast<float>(hi % 3 - 1), l4 = static_cast<float>(hi / 3 - 1);
       const float2 q = __ffma2_rn(make_float2(l3, l3), xv[3], __fmul2_rn(make_float2(l4, l4), xv[4]));
+      const float l = static_cast<float>(d2 - 1);
+      const float2 qc = __ffma2_rn(make_float2(l, l), xv[2], q);
+      const uint32_t row0 = col + static_cast<uint32_t>(9 * d2 + 27 * hi) * 256u;
 #pragma unroll
-      for (int d2 = 0; d2 < 3; ++d2) {
-        const float l = static_cast<float>(d2 - 1);
-        const float2 qc = __ffma2_rn(make_float2(l, l), xv[2], q);
-        const uint32_t row0 = col + static_cast<uint32_t>(9 * d2 + 27 * hi) * 256u;
-#pragma unroll
-        for (int m = 0; m < 9; ++m) sts_f2(row0 + m * 256u, __fadd2_rn(qc, ab[m]));
-      }
+      for (int m = 0; m < 9; ++m) sts_f2(row0 + m * 256u, __fadd2_rn(qc, ab[m]));
     }
     // byte values 243..255 never occur: zero rows keep them harmless
     for (int i = tid; i < 13 * 64; i += kThreads) {
@@ -462,10 +462,13 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
   build_table<FMT>(a, j, tbase, xs, tid);
 
   // This lane's word of each group, and (1-bit, 2-bit) its block's scales of four
-  // rows: lanes without a word (their table columns are zero) read word 0 and the
+  // rows. Lanes without a word (their table columns are zero) read the word of the
+  // first lane of their quarter-warp, which the shared-memory unit then serves in
+  // the same wavefront (word 0 would collide with another lane's banks), and the
   // slice's first block.
   const int wl = lane_word<FMT>(lane, nb);
-  const uint32_t woff = 16u * static_cast<uint32_t>(wl < 0 ? 0 : wl);
+  const int wq = lane_word<FMT>(lane & ~7, nb);
+  const uint32_t woff = 16u * static_cast<uint32_t>(wl >= 0 ? wl : (wq >= 0 ? wq : 0));
   const int sblk = wl < 0 ? 0 : (FMT == LBQ_SIGN1 ? (lane >> 2) : (lane >> 1));
   const uint32_t soff = kScaleOff + 8u * static_cast<uint32_t>(sblk);
   const uint32_t lanereg = tbase | static_cast<uint32_t>(lane * 4);
