@@ -334,35 +334,43 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
   } else if (warp == 1) {
     // ---------------- MMA issue: 8 instructions of K = 16 per weight stage, four per
-    // activation slab. The whole warp runs the loop (so descriptors stay
-    // warp-uniform); one elected lane issues.
-    const uint32_t idesc = idesc_f16_m128(a.tile_m);
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % kStagesTC;
+    // activation slab, all from lane 0. The issue path is kept short (an MMA of 128 x
+    // 256 x 16 takes 128 cycles; with descriptors rebuilt per instruction the loop
+    // took ~140 cycles an MMA whatever its size): the accumulator columns of the
+    // eight K steps are fixed (nacc divides 8), a slab's descriptor is built once and
+    // advanced by 32 bytes (+2 in its address field) per K step.
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16_m128(a.tile_m);
+      uint32_t dcol[8];
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) dcol[ks] = tmem + static_cast<uint32_t>((ks & (a.nacc - 1)) * a.tile_m);
       bool ok = true;
-      if (lane == 0) ok = mbar_wait(fullA + 8 * s, static_cast<uint32_t>(kb / kStagesTC) & 1, a.fault, kFaultMma);
-      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
-      const uint32_t ta = tmem + kTmemA + 64u * s;
+      for (int kb = 0; kb < nkb && ok; ++kb) {
+        const int s = kb % kStagesTC;
+        ok = mbar_wait(fullA + 8 * s, static_cast<uint32_t>(kb / kStagesTC) & 1, a.fault, kFaultMma);
+        if (!ok) break;
+        const uint32_t ta = tmem + kTmemA + 64u * s;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int sl = 2 * kb + h, sb_i = sl % kSlabs;
-        if (lane == 0) ok = mbar_wait(fullB + 8 * sb_i, static_cast<uint32_t>(sl / kSlabs) & 1, a.fault, kFaultMma);
-        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
-        tc_fence_after_sync();
-        const uint32_t sb = bstage(sb_i);
+        for (int h = 0; h < 2; ++h) {
+          const int sl = 2 * kb + h, sb_i = sl % kSlabs;
+          ok = mbar_wait(fullB + 8 * sb_i, static_cast<uint32_t>(sl / kSlabs) & 1, a.fault, kFaultMma);
+          if (!ok) break;
+          tc_fence_after_sync();
+          const uint64_t bdesc = sw128_desc(bstage(sb_i));
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {  // K = 16: 8 tensor-memory columns of A, 32 bytes of B
-          const int ks = 4 * h + k4;
-          const int i = kb * (kTileK / 16) + ks;  // MMA number; accumulator i % nacc
-          mma_f16_ts_warp(tmem + static_cast<uint32_t>((i & (a.nacc - 1)) * a.tile_m), ta + 8u * ks,
-                          sw128_desc(sb + 32u * k4), idesc, i >= a.nacc ? 1u : 0u);
+          for (int k4 = 0; k4 < 4; ++k4) {  // K = 16: 8 tensor-memory columns of A, 32 bytes of B
+            const int ks = 4 * h + k4;
+            // the first MMA into each accumulator overwrites it
+            mma_f16_ts(dcol[ks], ta + 8u * ks, bdesc + 2u * k4, idesc, (kb > 0 || ks >= a.nacc) ? 1u : 0u);
+          }
+          mma_commit(emptyB + 8 * sb_i);  // the slab is free once these MMAs are done
         }
-        mma_commit_warp(emptyB + 8 * sb_i);  // the slab is free once these MMAs are done
+        if (!ok) break;
+        mma_commit(emptyA + 8 * s);  // and the weight stage once all eight are
       }
-      if (!ok) break;
-      mma_commit_warp(emptyA + 8 * s);  // and the weight stage once all eight are
+      mma_commit(accum);  // the accumulator is complete once every MMA is done
     }
-    mma_commit_warp(accum);  // the accumulator is complete once every MMA is done
+    __syncwarp();
   } else if (warp == 2) {
     // ---------------- packed weights: 128 rows x 4 blocks per copy (rows past N read 0)
     if (lane == 0) {
