@@ -35,6 +35,7 @@
 // Every wait is bounded (see sm100_async.cuh).
 #include <cudaTypedefs.h>
 
+#include <type_traits>
 #include <utility>
 
 #include "sm100_async.cuh"
@@ -285,11 +286,17 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const uint32_t tslot = emptyR + 8 * kRawStages;
   auto bstage = [&](int s) { return s == 0 ? bstage0 : tab + kHighB + (s - 1) * kStageB; };
 
+  // MMA issuers: with eight accumulators (token tiles of at most 32) the eight K steps
+  // of a block split into two halves with disjoint accumulators, issued from two
+  // warps on different schedulers (warps 1 and 3): a small MMA costs its issuing
+  // scheduler ~45 cycles and more while decoder warps share it, about as long as the
+  // tensor core needs for it.
+  const int nissue = a.nacc == 8 ? 2 : 1;
   load_sel_table(tab, tid);
   if (tid == 0) {
     for (int s = 0; s < kStagesTC; ++s) {
       mbar_init(fullA + 8 * s, kDecoders / 32);  // every decoder warp arrives
-      mbar_init(emptyA + 8 * s, 1);         // the MMA commit arrives
+      mbar_init(emptyA + 8 * s, nissue);    // every MMA issuer's commit arrives
     }
     for (int s = 0; s < kSlabs; ++s) {
       mbar_init(fullB + 8 * s, 1);          // the activation TMA lane arrives (+ bytes)
@@ -299,7 +306,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_init(fullR + 8 * r, 1);          // the weight TMA lane arrives (+ bytes)
       mbar_init(emptyR + 8 * r, kDecoders / 32); // every decoder warp has read its rows
     }
-    mbar_init(accum, 1);
+    mbar_init(accum, nissue);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -332,14 +339,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         mbar_wait(fullB + 8 * (sl % kSlabs), static_cast<uint32_t>(sl / kSlabs) & 1,
                   a.fault, kFaultX, /*give_up_after_fault=*/false);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || (warp == 3 && nissue == 2)) {
     // ---------------- MMA issue: 8 instructions of K = 16 per weight stage, four per
-    // activation slab, all from lane 0. The issue path is kept short (an MMA of 128 x
-    // 256 x 16 takes 128 cycles; with descriptors rebuilt per instruction the loop
-    // took ~140 cycles an MMA whatever its size): the accumulator columns of the
-    // eight K steps are fixed (nacc divides 8), a slab's descriptor is built once and
-    // advanced by 32 bytes (+2 in its address field) per K step.
-    if (lane == 0) {
+    // activation slab, from lane 0 of warp 1 (or slab halves 0 / 1 from warps 1 / 3).
+    // The issue path is kept short (an MMA of 128 x 256 x 16 takes 128 cycles; with
+    // descriptors rebuilt per instruction the loop took ~140 cycles an MMA whatever
+    // its size): the accumulator columns of the eight K steps are fixed (nacc divides
+    // 8), a slab's descriptor is built once and advanced by 32 bytes (+2 in its
+    // address field) per K step.
+    // (the slab range is a compile-time constant of each variant: a runtime loop
+    // over it measurably slowed the issue of large MMAs)
+    auto issue = [&](auto h_lo_c, auto h_hi_c) {
+      constexpr int h_lo = decltype(h_lo_c)::value, h_hi = decltype(h_hi_c)::value;
       const uint32_t idesc = idesc_f16_m128(a.tile_m);
       uint32_t dcol[8];
 #pragma unroll
@@ -351,7 +362,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (!ok) break;
         const uint32_t ta = tmem + kTmemA + 64u * s;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = h_lo; h < h_hi; ++h) {
           const int sl = 2 * kb + h, sb_i = sl % kSlabs;
           ok = mbar_wait(fullB + 8 * sb_i, static_cast<uint32_t>(sl / kSlabs) & 1, a.fault, kFaultMma);
           if (!ok) break;
@@ -366,9 +377,17 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           mma_commit(emptyB + 8 * sb_i);  // the slab is free once these MMAs are done
         }
         if (!ok) break;
-        mma_commit(emptyA + 8 * s);  // and the weight stage once all eight are
+        mma_commit(emptyA + 8 * s);  // and the weight stage once every issuer's are
       }
       mma_commit(accum);  // the accumulator is complete once every MMA is done
+    };
+    if (lane == 0) {
+      using I0 = std::integral_constant<int, 0>;
+      using I1 = std::integral_constant<int, 1>;
+      using I2 = std::integral_constant<int, 2>;
+      if (nissue == 1) issue(I0{}, I2{});
+      else if (warp == 1) issue(I0{}, I1{});
+      else issue(I1{}, I2{});
     }
     __syncwarp();
   } else if (warp == 2) {

@@ -54,6 +54,21 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// The same with a suspend-time hint: a thread whose phase is not complete sleeps (up
+// to about `ns`) until it completes instead of returning at once, so waiting warps
+// do not take issue slots from working ones.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete. Gives up (returns false)
 // after kWaitLimitNs, recording `code` in *fault, or -- unless give_up_after_fault is
 // false -- as soon as another wait has already given up.
@@ -62,8 +77,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255) == 0) {
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    if ((i & 15) == 0) {
       if (give_up_after_fault && *reinterpret_cast<volatile unsigned*>(fault) != 0) return false;
       if (global_ns() - t0 > kWaitLimitNs) {
         atomicExch(fault, code);
