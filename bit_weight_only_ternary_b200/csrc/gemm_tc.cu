@@ -255,6 +255,12 @@ __device__ __forceinline__ void decode_quarter(const uint4 (&raw)[7], int r, uin
   }
 }
 
+// v * 2^e, exactly as ldexpf (one rounding): a multiply by the power of two when it
+// is a normal float, which is every row but those of extreme magnitude.
+__device__ __forceinline__ float scale_pow2(float v, int e) {
+  return (e >= -126 && e <= 127) ? v * __int_as_float((e + 127) << 23) : ldexpf(v, e);
+}
+
 __global__ void __launch_bounds__(kThreadsTC, 1)
     gemm_tern_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_w,
@@ -507,7 +513,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           // undo the activation row's power-of-two scaling (exact)
-          const float y = ldexpf(__uint_as_float(v[i]), xe[c0 + i]);
+          const float y = scale_pow2(__uint_as_float(v[i]), xe[c0 + i]);
           const uint32_t addr = ot + static_cast<uint32_t>((c0 + i) * 256 + rloc * 2);
           asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(f32_to_bf16_bits(y)) : "memory");
         }
@@ -537,7 +543,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           const int64_t m = m0 + c0 + i;
           if (m < a.M) {
             // undo the activation row's power-of-two scaling (exact)
-            const float y = ldexpf(__uint_as_float(v[i]), a.xexp[m]);
+            const float y = scale_pow2(__uint_as_float(v[i]), a.xexp[m]);
             if (a.part)
               a.part[(static_cast<int64_t>(blockIdx.z) * a.M + m) * a.N + ne] = y;
             else
