@@ -277,12 +277,15 @@ def test_ternary_gemm_tensor_cores(L, orc, M, N, K):
 
 
 def test_ternary_gemm_large_activations_are_scaled_into_fp16(L, orc):
-    """Rows of X beyond fp16's range (bf16 values up to 3e38 are finite) still come out right."""
-    M, N, K = 4, 128, 512
+    """Rows of X beyond fp16's range (bf16 values up to 3e38 are finite) still come out right,
+    including rows whose scale-back factor 2^e is itself outside fp32's normal range."""
+    M, N, K = 6, 128, 512
     W = synth.weights(N, K, 61)
     X = synth.activations(M, K, 62)
     X[1] *= 2.0 ** 40
     X[2] *= 2.0 ** -30
+    X[3] *= 2.0 ** -125   # e = ilogb(max|x|) - 14 < -126: the ldexpf branch
+    X[4] *= 2.0 ** 100    # large e, still a normal power of two
     pw, codes, scales = _pack_both(L, orc, TERN5, W)
     Yg = L.lbq_gemm(pw, X.cuda())
     Y, B = orc.gemm(TERN5, codes, scales, K, synth.bf16_bits(X), None)
