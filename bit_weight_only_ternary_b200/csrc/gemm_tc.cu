@@ -510,12 +510,37 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(u[i]));
         }
+        // the 16 tokens' exponents first (four 16-byte loads), then the 16 conversions,
+        // then the stores: interleaved, each store's memory clobber held the next
+        // exponent load behind it
+        int ex[16];
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) {
+          const int4 e4 = *reinterpret_cast<const int4*>(xe + c0 + i);
+          ex[i] = e4.x;
+          ex[i + 1] = e4.y;
+          ex[i + 2] = e4.z;
+          ex[i + 3] = e4.w;
+        }
+        // undo the activation rows' power-of-two scaling (exact): a multiply by 2^e
+        // unless some exponent of the chunk is outside fp32's normal range (a branch
+        // on the whole chunk: per element, the compiler evaluated ldexpf every time)
+        bool normal = true;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) normal = normal && ex[i] >= -126 && ex[i] <= 127;
+        uint16_t h[16];
+        if (normal) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            h[i] = f32_to_bf16_bits(__uint_as_float(v[i]) * __int_as_float((ex[i] + 127) << 23));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) h[i] = f32_to_bf16_bits(ldexpf(__uint_as_float(v[i]), ex[i]));
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          // undo the activation row's power-of-two scaling (exact)
-          const float y = scale_pow2(__uint_as_float(v[i]), xe[c0 + i]);
           const uint32_t addr = ot + static_cast<uint32_t>((c0 + i) * 256 + rloc * 2);
-          asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(f32_to_bf16_bits(y)) : "memory");
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(h[i]) : "memory");
         }
       }
       fence_proxy_async_smem();  // the generic-proxy writes, before the TMA reads them
