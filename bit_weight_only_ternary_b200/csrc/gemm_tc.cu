@@ -595,9 +595,19 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t* __restric
                                                         int* __restrict__ xexp) {
   __shared__ float red[8];
   const int64_t m = blockIdx.x;
-  const uint16_t* xr = X + m * K;
+  // 16-byte accesses: 8 values a thread (K is a multiple of 128, rows 16-byte aligned)
+  const uint4* xr = reinterpret_cast<const uint4*>(X + m * K);
+  uint4* hr = reinterpret_cast<uint4*>(Xh + m * K);
+  const int64_t K8 = K / 8;
+  auto lo = [](uint32_t w) { return __uint_as_float(w << 16); };
+  auto hi = [](uint32_t w) { return __uint_as_float(w & 0xffff0000u); };
   float mx = 0.0f;
-  for (int64_t k = threadIdx.x; k < K; k += blockDim.x) mx = fmaxf(mx, fabsf(bf16_bits_to_f32(xr[k])));
+  for (int64_t k = threadIdx.x; k < K8; k += blockDim.x) {
+    const uint4 v = xr[k];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) mx = fmaxf(mx, fmaxf(fabsf(lo(w[q])), fabsf(hi(w[q]))));
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
@@ -605,8 +615,28 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t* __restric
   mx = red[0];
   for (int i = 1; i < static_cast<int>(blockDim.x >> 5); ++i) mx = fmaxf(mx, red[i]);
   const int e = mx > 0.0f ? ilogbf(mx) - 14 : 0;  // floor(log2(max|x|)) - 14
-  for (int64_t k = threadIdx.x; k < K; k += blockDim.x)
-    Xh[m * K + k] = __half_as_ushort(__float2half_rn(ldexpf(bf16_bits_to_f32(xr[k]), -e)));
+  // x * 2^-e to fp16: a multiply by the power of two when it is a normal float (exact,
+  // as ldexpf), ldexpf otherwise
+  // (two loops: a select per element had the compiler evaluate ldexpf every time)
+  auto pack = [](float a0, float a1) {
+    return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(a0))) |
+           (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(a1))) << 16);
+  };
+  if (-e >= -126 && -e <= 127) {
+    const float f = __int_as_float((127 - e) << 23);
+    for (int64_t k = threadIdx.x; k < K8; k += blockDim.x) {
+      const uint4 v = xr[k];
+      hr[k] = make_uint4(pack(lo(v.x) * f, hi(v.x) * f), pack(lo(v.y) * f, hi(v.y) * f),
+                         pack(lo(v.z) * f, hi(v.z) * f), pack(lo(v.w) * f, hi(v.w) * f));
+    }
+  } else {
+    for (int64_t k = threadIdx.x; k < K8; k += blockDim.x) {
+      const uint4 v = xr[k];
+      auto sc = [&](float x) { return ldexpf(x, -e); };
+      hr[k] = make_uint4(pack(sc(lo(v.x)), sc(hi(v.x))), pack(sc(lo(v.y)), sc(hi(v.y))),
+                         pack(sc(lo(v.z)), sc(hi(v.z))), pack(sc(lo(v.w)), sc(hi(v.w))));
+    }
+  }
   if (threadIdx.x == 0) xexp[m] = e;
 }
 
