@@ -154,12 +154,13 @@ constexpr SelTable make_sel_table() {
 }
 __device__ const SelTable g_sel_table = make_sel_table();
 
-// Replicates the table into shared memory as [byte][even/odd][16 lane slots] x 8 bytes.
-__device__ __forceinline__ void load_sel_table(uint32_t tab, int tid) {
+// Replicates the table into shared memory as [byte][even/odd][16 lane slots] x 8 bytes
+// (thread d of n threads).
+__device__ __forceinline__ void load_sel_table(uint32_t tab, int d, int n) {
   const uint2* src = reinterpret_cast<const uint2*>(&g_sel_table);
   constexpr int kSlots = 243 * 2 * 16;
 #pragma unroll 4
-  for (int i = tid; i < kSlots; i += kThreadsTC) {
+  for (int i = d; i < kSlots; i += n) {
     const uint2 e = __ldg(src + (i >> 4));
     asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(tab + 8u * i), "r"(e.x), "r"(e.y) : "memory");
   }
@@ -298,7 +299,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   // scheduler ~45 cycles and more while decoder warps share it, about as long as the
   // tensor core needs for it.
   const int nissue = a.nacc == 8 ? 2 : 1;
-  load_sel_table(tab, tid);
   if (tid == 0) {
     for (int s = 0; s < kStagesTC; ++s) {
       mbar_init(fullA + 8 * s, kDecoders / 32);  // every decoder warp arrives
@@ -418,6 +418,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   } else if (warp >= 4) {
     // ---------------- decode: thread d owns row d % 128, quarter r = d / 128 of each block
     const int d = tid - 128;
+    // the selector table, loaded while the first weight copies are in flight
+    load_sel_table(tab, d, kDecoders);
+    named_bar_sync(2, kDecoders);
     const int row = d & (kTileN - 1), r4 = d >> 7;
     const uint32_t base_e = tab | (static_cast<uint32_t>(lane & 15) << 3), base_o = base_e + 128u;
     const uint32_t tlane = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + kTmemA + 16u * r4;
