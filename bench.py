@@ -45,8 +45,8 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 # four products, averaged per launch), keyed by the hash of the kernel source it was
 # taken on; reported as null once that source changes.
 NCU_TRAFFIC = {
-    # profiles/gemv_tern_1layer_full.md: 72.41 MB read + 2.6 KB written over the 4 launches
-    ("tern", "27026c9893bb8537"): 18.103e6,
+    # profiles/gemv_tern_1layer_full.md: 72.41 MB read + 512 B written over the 4 launches
+    ("tern", "679f5ead37a83e5b"): 18.102e6,
 }
 
 
@@ -275,8 +275,11 @@ def ours(args):
     roof["traffic"] = tr
     if M >= 512:
         tf = flops / (kern_ms * 1e-3) / 1e12
+        # frac against the burst peak; a pass of many products runs under the power cap,
+        # so the sustained peak is given beside it
         roof.update({"bound": "tensor", "achieved": round(tf, 1), "peak": tc_peak, "unit": "TFLOP/s",
-                     "frac": round(tf / tc_peak, 4)})
+                     "frac": round(tf / tc_peak, 4), "peak_sustained": tc_sust,
+                     "frac_of_sustained": round(tf / tc_sust, 4)})
 
     # ---- end to end: activations in from pinned host memory, outputs back, every step
     xin_host = torch.cat([p["X"].reshape(-1) for p in prods]).cpu().pin_memory()
