@@ -164,6 +164,20 @@ def build_layers(L, synth, fmt, M, n_layers, seed, device, torch):
     return prods
 
 
+def max_over_ranks(ms, world, dist, device, torch):
+    """The slowest rank's time: every rank takes part (same collective on all ranks)."""
+    if world <= 1:
+        return ms
+    tt = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def job_rate(world, units_per_rank, ms_step):
+    """Whole-job rate: the units all ranks processed per second of the slowest rank."""
+    return world * units_per_rank / (ms_step * 1e-3)
+
+
 def run_step(L, prods, D, ws, M):
     for p in prods:
         if M == 1:
@@ -236,14 +250,10 @@ def ours(args):
                 graph.replay()
             t1.record(stream)
         barrier()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dist, dev, torch)
     ms_step = ms / args.steps
-    gbs = world * weight_bytes / (ms_step * 1e-3) / 1e9
-    tok_s = world * M / (ms_step * 1e-3)
+    gbs = job_rate(world, weight_bytes, ms_step) / 1e9
+    tok_s = job_rate(world, M, ms_step)
 
     # ---- per-launch durations of the GEMV kernel (events between launches, queued ahead)
     per_launch_ms = []
@@ -310,14 +320,10 @@ def ours(args):
             g2.replay()
         t1.record(stream)
     barrier()
-    ems = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ems], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ems = float(tt.item())
+    ems = max_over_ranks(t0.elapsed_time(t1), world, dist, dev, torch)
     e_step = ems / e_steps
-    e2e = {"value": round(world * weight_bytes / (e_step * 1e-3) / 1e9, 1), "unit": "GB/s",
-           "tok_s_equiv": round(world * M / (e_step * 1e-3), 2),
+    e2e = {"value": round(job_rate(world, weight_bytes, e_step) / 1e9, 1), "unit": "GB/s",
+           "tok_s_equiv": round(job_rate(world, M, e_step), 2),
            "h2d_bytes_per_step": xin_host.numel() * 2, "d2h_bytes_per_step": y_host.numel() * 2}
 
     # ---- sampled parity of the timed configuration against the oracle (rank 0)
