@@ -39,7 +39,9 @@
 //    row range or after a meeting of the range's CTAs, measured slower: the tail of
 //    L2 round trips then runs on a handful of SMs.)
 //  * Programmatic dependent launch: the copy warp never waits for the previous
-//    kernel, so the ring fills while it finishes. Only the batch-1 kernels let
+//    kernel, so its first copies (one slot per warp group) land while it finishes;
+//    the other slots are filled once the table is built (their shared-memory writes
+//    slowed the build down). Only the batch-1 kernels let
 //    their successor start early, and they never write packed weights; any other
 //    kernel has completed before this one starts. x, y and the workspace are
 //    touched only after the wait.
@@ -67,7 +69,7 @@ constexpr uint32_t kXBytes = 4096;  // the slice of x as fp32 (up to 1024)
 constexpr int kMaxSlots = 32;
 // x and the mbarriers, rounded up so that the ring slots after them stay 128-byte
 // aligned, as tensor copies into shared memory require
-constexpr uint32_t kMisc = (kXBytes + 2 * 8 * kMaxSlots + 1023) & ~1023u;
+constexpr uint32_t kMisc = (kXBytes + 2 * 8 * kMaxSlots + 8 + 1023) & ~1023u;
 // 225 KB: with the 1 KB every CTA reserves, a CTA of the split-K sum kernel still
 // fits beside this one in the SM's 228 KB.
 constexpr uint32_t kSmem = 225 * 1024;
@@ -376,6 +378,7 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
   }
   float* xs = reinterpret_cast<float*>(smem + (misc - sbase));
   const uint32_t full0 = misc + kXBytes, empty0 = full0 + 8 * kMaxSlots;
+  const uint32_t built = empty0 + 8 * kMaxSlots;  // the table is built (inside kMisc)
   auto slot_addr = [&](int s) {
     return s < s_lo ? lo0 + static_cast<uint32_t>(s) * T::kSlot
                     : hi0 + static_cast<uint32_t>(s - s_lo) * T::kSlot;
@@ -385,6 +388,7 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, kSub);
     }
+    mbar_init(built, 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -420,9 +424,14 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
       const int32_t nslots = (n_units + kSub - 1) / kSub;
       int slot = 0;
       uint32_t round = 0;
+      int32_t issued = 0;
       for (int32_t q = 0; q < nslots; ++q) {
         const uint32_t full = full0 + 8 * slot;
         if (round > 0 && !mbar_wait(empty0 + 8 * slot, (round - 1) & 1, a.fault, kFaultRing)) break;
+        // one slot per warp group up front; the rest once the table is built, so that
+        // their shared-memory writes do not slow the build down
+        if (q == kGroups && !mbar_wait(built, 0, a.fault, kFaultRing)) break;
+        ++issued;
         const uint32_t dst = slot_addr(slot);
         const int32_t u0 = kSub * q;
         const int32_t nu = n_units - u0 < kSub ? n_units - u0 : kSub;
@@ -443,6 +452,11 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
           ++round;
         }
       }
+      // Every issued copy lands before the CTA can exit (after a fault the consumers
+      // may have stopped taking them): the last fill of each slot, bounded.
+      for (int32_t q = issued - S > 0 ? issued - S : 0; q < issued; ++q)
+        mbar_wait(full0 + 8 * (q % S), static_cast<uint32_t>(q / S) & 1, a.fault, kFaultRing,
+                  /*give_up_after_fault=*/false);
     }
     return;  // the consumers synchronise among themselves from here on
   }
@@ -460,6 +474,7 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
   x_store<FMT>(x_issue<FMT>(a, j, tid), xs, tid);
   named_bar_sync(1, kThreads);
   build_table<FMT>(a, j, tbase, xs, tid);
+  if (tid == 0) mbar_arrive(built);
 
   // This lane's word of each group, and (1-bit, 2-bit) its block's scales of four
   // rows. Lanes without a word (their table columns are zero) read the word of the
