@@ -173,6 +173,11 @@ size_t lbq_workspace_bytes(const lbq_weights* w, int64_t M);
  * weights; for LBQ_Q2RHT the input is first rotated, y = W_hat (H D x / sqrt 512),
  * with D from lbq_rht_signs (NULL for other formats). fp32 accumulation; y is
  * rounded to bf16 once, at the end. Workspace as lbq_workspace_bytes(w, 1).
+ * Ordering: the product starts early beside the previous kernel of the stream
+ * (programmatic dependent launch) and touches x, y and the workspace only once that
+ * kernel has finished, but it reads the packed weights at once. Weights written on
+ * the same stream are therefore safe as long as the writing kernel does not itself
+ * let its successor start early: lbq_pack, copies and ordinary kernels do not.
  * Errors: LBQ_ERR_ARG (nulls, D missing for Q2RHT), LBQ_ERR_SHAPE, LBQ_ERR_ALIGN,
  * LBQ_ERR_FORMAT, LBQ_ERR_WORKSPACE, LBQ_ERR_CUDA. */
 lbq_status lbq_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D, uint16_t* y,
