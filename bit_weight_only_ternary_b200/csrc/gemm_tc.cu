@@ -116,13 +116,6 @@ __device__ __forceinline__ uint32_t idesc_f16_m128(int n) {
   return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
 }
 
-__device__ __forceinline__ uint4 lds_u128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
-  return v;
-}
 // ---------------------------------------------------------------- byte -> fp16 values
 // A byte v = d0 + 3 d1 + 9 d2 + 27 d3 + 81 d4 holds five digits d = t + 1 (weights
 // 5j .. 5j + 4 of the block for byte j). A register V = (s, -s) as two fp16, next

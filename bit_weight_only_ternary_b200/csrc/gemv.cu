@@ -127,11 +127,8 @@ __device__ __forceinline__ int digit_weight(int slot, int l, int e, int nb) {
 }
 
 template <int FMT>
+// The packed weights reach the kernel as tensor maps (see the launch).
 struct Args {
-  const uint8_t* codes;
-  const uint16_t* scales;
-  int64_t cstride;  // code bytes per row (a group of four rows is 4 * cstride)
-  int64_t sstride;  // scales per row
   int64_t K, N;
   const uint16_t* x;
   const int8_t* D;
@@ -140,7 +137,7 @@ struct Args {
   int KS;           // number of slices
   int G;            // CTAs per slice
   int nblk;         // scale blocks per row
-  unsigned* fault;  // set when the shared-memory layout check fails
+  unsigned* fault;  // the device fault word (layout check, bounded waits)
 };
 
 __device__ __forceinline__ void sts_f2(uint32_t addr, float2 v) {
@@ -657,10 +654,6 @@ cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uin
     configured[dev] = true;
   }
   Args<FMT> a;
-  a.codes = static_cast<const uint8_t*>(w->codes);
-  a.scales = static_cast<const uint16_t*>(w->scales);
-  a.cstride = w->code_stride;
-  a.sstride = w->scale_stride;
   a.K = w->K;
   a.N = w->N;
   a.x = x;
