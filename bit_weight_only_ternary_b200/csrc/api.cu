@@ -69,6 +69,7 @@ const char* lbq_status_string(lbq_status st) {
     case LBQ_ERR_FORMAT: return "unknown packed format";
     case LBQ_ERR_CUDA: return "CUDA error";
     case LBQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case LBQ_ERR_DEVICE_WAIT: return "a bounded wait inside a kernel gave up";
     default: return "unknown status";
   }
 }
@@ -134,8 +135,10 @@ lbq_status lbq_device_fault(uint32_t* code) {
   if (cudaMemcpy(&v, word, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return LBQ_ERR_CUDA;
   if (v && cudaMemset(word, 0, sizeof(v)) != cudaSuccess) return LBQ_ERR_CUDA;
   *code = v;
-  return LBQ_OK;
+  return v ? LBQ_ERR_DEVICE_WAIT : LBQ_OK;
 }
+
+lbq_status lbq_selftest_wait(void* stream) { return from_cuda(lbq_launch_wait_selftest(as_stream(stream))); }
 
 size_t lbq_workspace_bytes(const lbq_weights* w, int64_t M) {
   Layout L;

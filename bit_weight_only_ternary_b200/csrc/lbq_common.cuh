@@ -114,6 +114,8 @@ cudaError_t lbq_launch_hadamard(const uint16_t* x, const int8_t* D, int64_t M, i
 size_t lbq_gemv_workspace(const lbq_weights* w);
 // Device address of the word bounded device waits report to (current device), or NULL.
 unsigned* lbq_fault_word();
+// Launches the kernel whose bounded wait runs out on purpose (selftest.cu).
+cudaError_t lbq_launch_wait_selftest(cudaStream_t s);
 cudaError_t lbq_launch_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D,
                             uint16_t* y, void* ws, cudaStream_t s);
 size_t lbq_gemm_workspace(const lbq_weights* w, int64_t M);

@@ -73,14 +73,15 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 // after kWaitLimitNs, recording `code` in *fault, or -- unless give_up_after_fault is
 // false -- as soon as another wait has already given up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* fault,
-                                          unsigned code, bool give_up_after_fault = true) {
+                                          unsigned code, bool give_up_after_fault = true,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
     if ((i & 15) == 0) {
       if (give_up_after_fault && *reinterpret_cast<volatile unsigned*>(fault) != 0) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit_ns) {
         atomicExch(fault, code);
         return false;
       }

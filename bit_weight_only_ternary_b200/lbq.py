@@ -21,7 +21,8 @@ LBQ_OK, LBQ_ERR_ARG, LBQ_ERR_SHAPE, LBQ_ERR_ALIGN, LBQ_ERR_FORMAT, LBQ_ERR_CUDA,
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblbq.so")
 EXPORTS = ("lbq_status_string", "lbq_packed_layout", "lbq_pack", "lbq_unpack", "lbq_rht_signs",
-           "lbq_hadamard", "lbq_workspace_bytes", "lbq_gemv", "lbq_gemm", "lbq_gemv_noalloc", "lbq_device_fault")
+           "lbq_hadamard", "lbq_workspace_bytes", "lbq_gemv", "lbq_gemm", "lbq_gemv_noalloc", "lbq_device_fault",
+           "lbq_selftest_wait")
 LBQ_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -56,6 +57,7 @@ def _load():
         "lbq_gemm": (ctypes.c_int, [W, p, i64, p, p, p, sz, p]),
         "lbq_gemv_noalloc": (ctypes.c_int, [W, p, p, p, p]),
         "lbq_device_fault": (ctypes.c_int, [p]),
+        "lbq_selftest_wait": (ctypes.c_int, [p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -162,8 +164,15 @@ def lbq_hadamard(x: torch.Tensor, D: torch.Tensor, out=None, stream=None) -> tor
 def lbq_device_fault() -> int:
     """Code of a bounded in-kernel wait that gave up since the last query (0: none)."""
     code = ctypes.c_uint32()
-    _check(_lib.lbq_device_fault(ctypes.byref(code)), "lbq_device_fault")
+    st = _lib.lbq_device_fault(ctypes.byref(code))
+    if st != LBQ_ERR_DEVICE_WAIT:
+        _check(st, "lbq_device_fault")
     return code.value
+
+
+def lbq_selftest_wait(stream=None) -> None:
+    """Enqueues the kernel whose bounded wait runs out on purpose (fault code 11)."""
+    _check(_lib.lbq_selftest_wait(_stream(stream)), "lbq_selftest_wait")
 
 
 def lbq_workspace_bytes(pw: PackedWeights, M: int = 1) -> int:

@@ -199,10 +199,17 @@ lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const in
  * kernels (on an mbarrier, for a TMA copy or a slot) is bounded by about 2 s; a
  * wait that runs out records a non-zero *code (3: shared-memory layout of the
  * batch-1 product, 4-9: tensor-core product stages, 10: the batch-1 product's
- * weight copies) and the kernel returns early
- * with incomplete outputs instead of hanging. A non-zero code means a library fault. Synchronises the device.
- * Errors: LBQ_ERR_ARG (code NULL), LBQ_ERR_CUDA. */
+ * weight copies, 11: lbq_selftest_wait) and the kernel returns early with
+ * incomplete outputs instead of hanging. Synchronises the device.
+ * Returns LBQ_OK with *code = 0 when no wait gave up, LBQ_ERR_DEVICE_WAIT with the
+ * code otherwise. Errors: LBQ_ERR_ARG (code NULL), LBQ_ERR_CUDA. */
 lbq_status lbq_device_fault(uint32_t* code);
+
+/* Test hook for the path above: enqueues a kernel whose one bounded wait (on an
+ * mbarrier nothing arrives on, limited to 20 ms) runs out, records code 11 and
+ * returns. The device stays usable; the next lbq_device_fault reports and clears it.
+ * Errors: LBQ_ERR_CUDA. */
+lbq_status lbq_selftest_wait(void* stream);
 
 /* lbq_gemv without a workspace argument, for callers that cannot allocate device
  * memory: a host that reaches the library only through this C interface and has no

@@ -303,3 +303,21 @@ def test_ternary_gemm_27b_gate_up_sampled(L, orc):
     codes, scales = orc.pack(TERN5, Wd[rows].cpu().numpy())
     Y, B = orc.gemm(TERN5, codes, scales, K, synth.bf16_bits(X), None, nthreads=NTHREADS)
     _check_products(Yg[:, rows], Y, B, "27B gate+up, M=512")
+
+
+def test_bounded_wait_gives_up_and_device_stays_usable(L, orc):
+    """A kernel wait that runs out (an mbarrier nothing arrives on, 20 ms limit) records
+    its code, returns instead of hanging, and the next product still runs correctly."""
+    assert L.lbq_device_fault() == 0
+    L.lbq_selftest_wait()
+    torch.cuda.synchronize()
+    assert L.lbq_device_fault() == 11
+    assert L.lbq_device_fault() == 0  # the record is cleared by the query
+    N, K = 64, 1024
+    W = synth.weights(N, K, 91)
+    x = synth.activations(1, K, 92)
+    pw, codes, scales = _pack_both(L, orc, TERN5, W)
+    y = L.lbq_gemv(pw, x[0].cuda())
+    Y, B = orc.gemm(TERN5, codes, scales, K, synth.bf16_bits(x), None)
+    _check_products(y, Y[0], B[0], "after a timed-out wait")
+    assert L.lbq_device_fault() == 0
