@@ -14,6 +14,19 @@ inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 inline lbq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LBQ_OK : LBQ_ERR_CUDA; }
 
+// Up to kTernPerTokenMaxM tokens a ternary product runs as one batch-1 product per
+// token: on the tensor cores a 16-token tile costs about as much as a 2-token one
+// (each N = 16 MMA is bound by its issue, not by its work), ~125 us per 27B-shaped
+// layer, while a batch-1 product costs ~38 us per layer and token (measured: at 8
+// tokens the per-token products took 2.4 times as long as the tensor cores).
+constexpr int64_t kTernPerTokenMaxM = 3;
+
+inline bool per_token(const lbq_weights* w, int64_t M) {
+  if (M == 1) return true;
+  return w->fmt == LBQ_TERN5 && M <= kTernPerTokenMaxM &&
+         !(lbq_gemv_workspace(w) && w->N > lbq::kMaxSplitRows);
+}
+
 inline bool fmt_known(int32_t fmt) {
   return fmt == LBQ_TERN5 || fmt == LBQ_SIGN1 || fmt == LBQ_Q2RHT;
 }
@@ -143,7 +156,7 @@ lbq_status lbq_selftest_wait(void* stream) { return from_cuda(lbq_launch_wait_se
 size_t lbq_workspace_bytes(const lbq_weights* w, int64_t M) {
   Layout L;
   if (check_weights(w, &L) != LBQ_OK || M < 1) return 0;
-  return M == 1 ? lbq_gemv_workspace(w) : lbq_gemm_workspace(w, M);
+  return per_token(w, M) ? lbq_gemv_workspace(w) : lbq_gemm_workspace(w, M);
 }
 
 lbq_status lbq_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D, uint16_t* y,
@@ -160,9 +173,15 @@ lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const in
   Layout L;
   lbq_status st = check_product(w, X, M, D, Y, workspace, workspace_bytes, &L);
   if (st != LBQ_OK) return st;
-  if (M == 1) {
+  if (per_token(w, M)) {
     if (lbq_gemv_workspace(w) && w->N > lbq::kMaxSplitRows) return LBQ_ERR_SHAPE;
-    return from_cuda(lbq_launch_gemv(w, X, D, Y, workspace, as_stream(stream)));
+    // one batch-1 product per token, in stream order (they share the workspace)
+    for (int64_t m = 0; m < M; ++m) {
+      const cudaError_t e =
+          lbq_launch_gemv(w, X + m * w->K, D, Y + m * w->N, workspace, as_stream(stream));
+      if (e != cudaSuccess) return LBQ_ERR_CUDA;
+    }
+    return LBQ_OK;
   }
   return from_cuda(lbq_launch_gemm(w, X, M, D, Y, workspace, as_stream(stream)));
 }

@@ -184,10 +184,13 @@ lbq_status lbq_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D, ui
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* Batched product Y[m][n] = sum_k W_hat[n][k] X[m][k] for M rows of bf16 X
- * ([M][K], row stride K) into bf16 Y ([M][N], row stride N). Small M streams the
- * weights once for all M rows; large M dequantises weight tiles into shared
- * memory and runs tcgen05 bf16 MMA with fp32 accumulation in tensor memory.
- * Same formats, D and workspace rules as lbq_gemv (workspace for this M). */
+ * ([M][K], row stride K) into bf16 Y ([M][N], row stride N). Ternary weights:
+ * up to 3 rows run as one batch-1 product per row (lbq_gemv's kernels, in stream
+ * order), more rows dequantise weight tiles into tensor memory and run tcgen05
+ * fp16 MMAs with fp32 accumulation (the activations are scaled into fp16 by an exact
+ * power of two per row). 1-bit and 2-bit weights: a CUDA-core kernel that streams
+ * the weights once for up to 8 rows at a time. Same formats, D and workspace rules
+ * as lbq_gemv (workspace for this M, from lbq_workspace_bytes). */
 lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const int8_t* D,
                     uint16_t* Y, void* workspace, size_t workspace_bytes, void* stream);
 

@@ -178,7 +178,7 @@ def test_gemv_one_27b_layer(L, orc, fmt):
 
 
 @pytest.mark.parametrize("fmt", FMTS)
-@pytest.mark.parametrize("M", (2, 8, 32, 100))
+@pytest.mark.parametrize("M", (2, 8, 13, 32, 100))
 def test_gemm_parity(L, orc, fmt, M):
     N, K = 384, 1536
     W = synth.weights(N, K, 4000 + M)
@@ -264,10 +264,11 @@ def test_no_bounded_device_wait_gave_up(L):
     assert L.lbq_device_fault() == 0
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 256, 1024), (3, 130, 640), (16, 128, 128), (128, 384, 1024),
-                                   (512, 256, 5120), (200, 1000, 2048)])
+@pytest.mark.parametrize("M,N,K", [(1, 256, 1024), (3, 130, 640), (13, 130, 640), (16, 128, 128),
+                                   (128, 384, 1024), (512, 256, 5120), (200, 1000, 2048)])
 def test_ternary_gemm_tensor_cores(L, orc, M, N, K):
-    """The tensor-core ternary product: ragged M and N, K from one block to 40."""
+    """The ternary product: ragged M and N, K from one block to 40 (M <= 3 runs one
+    batch-1 product per row, larger M the tensor cores)."""
     W = synth.weights(N, K, 6000 + M + N)
     X = synth.activations(M, K, 7000 + M)
     pw, codes, scales = _pack_both(L, orc, TERN5, W)
