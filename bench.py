@@ -46,7 +46,7 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 # taken on; reported as null once that source changes.
 NCU_TRAFFIC = {
     # profiles/gemv_tern_1layer_full.md: 72.42 MB read + 256 B written over the 4 launches
-    ("tern", "2d1bf45171d55708"): 18.104e6,
+    ("tern", "6a683c1dec9b0cc5"): 18.104e6,
 }
 
 
@@ -82,14 +82,28 @@ GEMV_SOURCES = ("gemv.cu", "rht.cuh", "sm100_async.cuh", "lbq_common.cuh")
 GEMM_SOURCES = ("gemm.cu", "gemm_tc.cu", "sm100_async.cuh", "lbq_common.cuh")
 
 
+def _code_only(text):
+    """The source without // comments and blank lines (comment edits keep the key)."""
+    out = []
+    for line in text.splitlines():
+        i = line.find("//")
+        while i >= 0 and line[:i].count('"') % 2 == 1:  # inside a string literal
+            i = line.find("//", i + 2)
+        code = (line if i < 0 else line[:i]).rstrip()
+        if code:
+            out.append(code)
+    return "\n".join(out)
+
+
 def kernel_source_hash(files=GEMV_SOURCES):
-    """Hash of the kernel sources a workload runs (keys the recorded ncu traffic)."""
+    """Hash of the kernel sources a workload runs, comments aside (keys the recorded
+    ncu traffic: a figure stands only for the code it was measured on)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_weight_only_ternary_b200", "csrc")
     for f in files:
         p = os.path.join(csrc, f)
         if os.path.exists(p):
-            h.update(open(p, "rb").read())
+            h.update(_code_only(open(p).read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -31,20 +31,21 @@
 //    cost more than the selects: measured.)
 //  * Scales. Ternary scales live in word 6 of each 28-byte block: lanes are mapped
 //    so that block b is lanes 8b .. 8b+6, and lane 8b+6 hands each pair of rows'
-//    scales to its block's lanes with one shuffle. 1-bit and 2-bit scales come
-//    with one 8-byte load per lane per four rows (group-of-four scale order).
+//    scales to its block's lanes with one shuffle. 1-bit and 2-bit scales come in
+//    the same tensor copies as the codes (group-of-four scale order): one 8-byte
+//    shared load per lane per four rows.
 //  * Split-K. Slices are spread over CTAs; slice sums go to the workspace and a
 //    small second kernel adds each row's slice sums in a fixed order and writes bf16
-//    y: results are deterministic. (Folding that sum into the main kernel, by the last CTA of a
-//    row range or after a meeting of the range's CTAs, measured slower: the tail of
-//    L2 round trips then runs on a handful of SMs.)
+//    y: results are deterministic. (Folding that sum into the main kernel, by the
+//    last CTA of a row range or after a meeting of the range's CTAs, measured slower:
+//    the tail of L2 round trips then runs on a handful of SMs. So did starting the
+//    sum of a row range as soon as its CTAs had counted themselves in.)
 //  * Programmatic dependent launch: the copy warp never waits for the previous
 //    kernel, so its first copies (one slot per warp group) land while it finishes;
 //    the other slots are filled once the table is built (their shared-memory writes
-//    slowed the build down). Only the batch-1 kernels let
-//    their successor start early, and they never write packed weights; any other
-//    kernel has completed before this one starts. x, y and the workspace are
-//    touched only after the wait.
+//    slowed the build down). Only the batch-1 kernels let their successor start
+//    early, and they never write packed weights; any other kernel has completed
+//    before this one starts. x, y and the workspace are touched only after the wait.
 #include <type_traits>
 
 #include "rht.cuh"
