@@ -161,6 +161,19 @@ def test_gemv_parity(L, orc, fmt, N, K):
     _check_products(y, Y[0], B[0], f"fmt {fmt} {N}x{K}")
 
 
+@pytest.mark.parametrize("fmt", (TERN5, SIGN1))
+@pytest.mark.parametrize("N,K", [(17, 1152), (130, 640), (1, 128)])
+def test_gemv_partial_last_slice(L, orc, fmt, N, K):
+    """K whose last slice holds fewer blocks than a full one (an odd number for the
+    1-bit format: its scale copy rounds up into the row's padding), ragged N."""
+    W = synth.weights(N, K, 2100 + N + K)
+    x = synth.activations(1, K, 3100 + K)
+    pw, codes, scales = _pack_both(L, orc, fmt, W)
+    y = L.lbq_gemv(pw, x[0].cuda())
+    Y, B = orc.gemm(fmt, codes, scales, K, synth.bf16_bits(x), None)
+    _check_products(y, Y[0], B[0], f"fmt {fmt} {N}x{K}")
+
+
 @pytest.mark.parametrize("fmt", FMTS)
 def test_gemv_one_27b_layer(L, orc, fmt):
     """Every output of one 27B-shaped layer (QKV, O, gate+up, down), full oracle check."""
