@@ -13,11 +13,13 @@
 // scaling (exact) that keeps every row inside fp16's range; the output is scaled
 // back exactly before the bf16 rounding.
 //
-// Tile: 128 weight rows (the MMA's M) x up to 128 tokens (the MMA's N; small batches
-// use N = 16 or 32) x 128 K per stage (one ternary block). Weights: fp16 in tensor
-// memory; activations: fp16 in shared memory. Warp roles:
+// Tile: 128 weight rows (the MMA's M) x up to 256 tokens (the MMA's N, a multiple of
+// 16 chosen by the tile planner) x 128 K per stage (one ternary block). Weights: fp16
+// in tensor memory; activations: fp16 in shared memory. Warp roles:
 //   warp 0   one lane streams fp16 activation tiles with 2D TMA (128-byte swizzle)
 //   warp 1   allocates tensor memory; one lane issues the MMAs and commits stages
+//   warp 3   for token tiles of at most 32: one lane issues the second half of each
+//            block's MMAs (into accumulators of its own)
 //   warp 2   one lane streams the packed weight rows with 2D TMA, four blocks
 //            (112 bytes) of 128 rows per copy
 //   warps 4-19 four threads per weight row, one per 32-weight quarter of each block.
@@ -31,7 +33,9 @@
 //            (tcgen05.st: the MMA reads the weight operand from tensor memory;
 //            a block's store completes while the next block is decoded); then the
 //            same warps read the accumulator (warp w reads lane quarter w % 4, the
-//            four warp groups split the columns) and write bf16 Y.
+//            four warp groups split the columns), undo the activation rows' scaling
+//            and stage bf16 Y in shared memory for one TMA store. They also load
+//            the selector table, once the first weight copies are in flight.
 // Every wait is bounded (see sm100_async.cuh).
 #include <cudaTypedefs.h>
 
