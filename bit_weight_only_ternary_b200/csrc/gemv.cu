@@ -22,7 +22,8 @@
 //    a time (7 to 10 KB) into a ring of shared-memory slots; the 16 compute warps
 //    take one unit each and read their lane's word of four rows with one 16-byte
 //    shared load per group. (Per-unit copies, 1.8 KB each, streamed at half the
-//    rate: the copy engine keeps few copies in flight. Loads into registers
+//    rate: the copy engine keeps few copies in flight. Eight-unit ternary copies
+//    measured the same as four-unit ones over a 16-layer pass. Loads into registers
 //    instead queue in the L1 path ahead of the x slice and the table build.)
 //  * Reduction. Each lane holds one word's partial sum for each of 16 rows; a
 //    transpose-reduce butterfly (16 shuffles) leaves row l's slice sum in lane l.
