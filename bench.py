@@ -34,12 +34,20 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 WORKLOADS = {
-    # name: (format, M)
-    "tern": (1, 1), "sign": (2, 1), "q2": (3, 1),
+    # name: (format, M); format 0: a mixed-format layer (see product_fmt)
+    "tern": (1, 1), "sign": (2, 1), "q2": (3, 1), "mixed": (0, 1),
     "gemm8": (1, 8), "gemm32": (1, 32), "gemm512": (1, 512), "gemm4096": (1, 4096),
 }
 FMT_NAME = {1: "ternary 5 trits/byte + fp16 scale per 128", 2: "1-bit sign + fp16 scale per 128",
-            3: "2-bit 4-level + fp16 scale per 32, input rotated by 512-point RHT"}
+            3: "2-bit 4-level + fp16 scale per 32, input rotated by 512-point RHT",
+            0: "mixed: attention (QKV, O) 2-bit + RHT, FFN (gate+up, down) ternary"}
+
+
+def product_fmt(fmt, mi):
+    """The format of product mi (0 QKV, 1 O, 2 gate+up, 3 down) of a layer."""
+    if fmt != 0:
+        return fmt
+    return 3 if mi < 2 else 1  # the mixed layer: 2-bit attention, ternary FFN
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 # dram bytes per launch of the dominant kernel from one ncu capture (one 27B layer, the
 # four products, averaged per launch), keyed by the hash of the kernel source it was
@@ -169,12 +177,12 @@ def build_layers(L, synth, fmt, M, n_layers, seed, device, torch):
     for layer in range(n_layers):
         for mi, (name, K, N) in enumerate(synth.LAYER_SHAPES):
             W = synth.weights(N, K, synth.seed_of(seed * 1000, layer, mi), device=device)
-            pw = L.lbq_pack(fmt, W)
+            pw = L.lbq_pack(product_fmt(fmt, mi), W)
             del W
             X = synth.activations(M, K, synth.seed_of(seed * 1000 + 500, layer, mi), device=device)
             Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
             prods.append({"layer": layer, "mi": mi, "name": name, "K": K, "N": N, "pw": pw,
-                          "X": X, "Y": Y})
+                          "X": X, "Y": Y, "fmt": product_fmt(fmt, mi)})
     return prods
 
 
@@ -194,10 +202,11 @@ def job_rate(world, units_per_rank, ms_step):
 
 def run_step(L, prods, D, ws, M):
     for p in prods:
+        Dp = D.get(p["K"]) if p["fmt"] == 3 else None
         if M == 1:
-            L.lbq_gemv(p["pw"], p["X"][0], D.get(p["K"]), p["Y"][0], ws)
+            L.lbq_gemv(p["pw"], p["X"][0], Dp, p["Y"][0], ws)
         else:
-            L.lbq_gemm(p["pw"], p["X"], D.get(p["K"]), p["Y"], ws)
+            L.lbq_gemm(p["pw"], p["X"], Dp, p["Y"], ws)
 
 
 def ours(args):
@@ -221,7 +230,7 @@ def ours(args):
     fmt, M = WORKLOADS[args.workload]
     prods = build_layers(L, synth, fmt, M, args.layers, args.seed + 7919 * rank, dev, torch)
     D = {}
-    if fmt == L.LBQ_Q2RHT:
+    if any(p["fmt"] == L.LBQ_Q2RHT for p in prods):
         for K in (synth.HIDDEN, synth.FFN):
             D[K] = L.lbq_rht_signs(args.seed * 31 + K, K, dev)
     ws_bytes = max(L.lbq_workspace_bytes(p["pw"], M) for p in prods)
@@ -242,8 +251,8 @@ def ours(args):
         with torch.cuda.graph(graph, stream=stream):
             run_step(L, prods, D, ws, M)
     # kernels per product: the GEMV, plus the split-K sum when K spans several slices
-    per_slice = 1024 if fmt == L.LBQ_SIGN1 else 512
-    launches = sum(1 + (p["K"] > per_slice) for p in prods) if M == 1 else len(prods)
+    launches = (sum(1 + (p["K"] > (1024 if p["fmt"] == L.LBQ_SIGN1 else 512)) for p in prods)
+                if M == 1 else len(prods))
     with torch.cuda.stream(stream):  # replays run on the stream the events are recorded on
         for _ in range(args.warmup):
             graph.replay()
@@ -343,7 +352,7 @@ def ours(args):
     # ---- sampled parity of the timed configuration against the oracle (rank 0)
     parity = None
     if rank == 0 and not args.no_parity:
-        parity = sampled_parity(L, synth, prods, fmt, M, D, ws, args, dev, torch)
+        parity = sampled_parity(L, synth, prods, M, D, ws, args, dev, torch)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -379,7 +388,7 @@ def ours(args):
     print(json.dumps(line), flush=True)
 
 
-def sampled_parity(L, synth, prods, fmt, M, D, ws, args, dev, torch):
+def sampled_parity(L, synth, prods, M, D, ws, args, dev, torch):
     """Re-draws a few timed matrices' weights, checks sampled output rows with the oracle."""
     import numpy as np
 
@@ -388,6 +397,7 @@ def sampled_parity(L, synth, prods, fmt, M, D, ws, args, dev, torch):
     picks = [prods[0], prods[1], prods[2], prods[-1]]
     rng = np.random.default_rng(0)
     for p in picks:
+        fmt = p["fmt"]
         run_step(L, [p], D, ws, M)
         torch.cuda.synchronize()
         W = synth.weights(p["N"], p["K"], synth.seed_of(args.seed * 1000, p["layer"], p["mi"]),
@@ -427,20 +437,22 @@ def cpu_baseline(args, fmt, M, budget_s=None):
     for mi, (name, K, N) in enumerate(synth.LAYER_SHAPES):
         n = max(threads, int(N * 0.02))
         W = synth.weights(n, K, 777 + mi).numpy()
-        codes, scales = oracle.pack(fmt, W)
+        f = product_fmt(fmt, mi)
+        codes, scales = oracle.pack(f, W)
         X = synth.bf16_bits(synth.activations(min(M, 8), K, 888 + mi))
-        D = oracle.rht_signs(5, K) if fmt == 3 else None
-        packed.append((K, n, codes, scales, X, D))
+        D = oracle.rht_signs(5, K) if f == 3 else None
+        packed.append((f, K, n, codes, scales, X, D))
     # time one pass over the sample, then repeat to fill the budget
     reps, elapsed = 0, 0.0
     t0 = time.perf_counter()
     while elapsed < budget_s or reps == 0:
-        for K, n, codes, scales, X, D in packed:
-            oracle.gemm(fmt, codes, scales, K, X, D, nthreads=threads)
+        for f, K, n, codes, scales, X, D in packed:
+            oracle.gemm(f, codes, scales, K, X, D, nthreads=threads)
         reps += 1
         elapsed = time.perf_counter() - t0
-    w_per_pass = sum(K * n for K, n, *_ in packed)
-    bytes_per_w = {1: 28 / 128, 2: 18 / 128, 3: 10 / 32}[fmt]
+    w_per_pass = sum(K * n for _, K, n, *_ in packed)
+    bpw = {1: 28 / 128, 2: 18 / 128, 3: 10 / 32}
+    bytes_per_w = sum(bpw[f] * K * n for f, K, n, *_ in packed) / w_per_pass
     m_eff = min(M, 8)
     w_per_s = w_per_pass * reps / elapsed          # weights x (m_eff activation rows) per second
     gbs = w_per_s * bytes_per_w / 1e9 * m_eff / M  # packed-weight bytes per second at M rows
