@@ -369,7 +369,9 @@ def ours(args):
         "metric": "packed-weight HBM GB/s (% of peak) & tok/s-equiv, batch-1 27B-shape GEMV",
         "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 x, fp32 accumulate, packed weights",
+        "scaling": "weak", "vs_baseline": None,
+        # the arithmetic: fp32 lookups and sums, or fp16 tensor-core MMAs into fp32
+        "dtype": "f32" if M <= 3 or fmt != 1 else "f16 (f32 accumulate)",
         "data": "synthetic (seeded N(0,0.02) weights, N(0,1) bf16 activations)",
         "tok_s_equiv": round(tok_s, 2), "pct_of_hbm_peak": round(100 * gbs / world / hbm_peak, 2),
         "config": {"workload": f"{args.layers} x 27B-shaped decoder layers (QKV 5120x7168, "
@@ -472,7 +474,7 @@ def reference(args):
     line = {"metric": "packed-weight HBM GB/s (% of peak) & tok/s-equiv, batch-1 27B-shape GEMV",
             "value": cpu["value"], "unit": "GB/s", "impl": "reference", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "fp64 (oracle)", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "tok_s_equiv": cpu["tok_s_equiv"],
             "config": {"workload": f"64 x 27B-shaped decoder layers, {FMT_NAME[fmt]}, M={M}",
                        "format": args.workload, "M": M},
