@@ -44,3 +44,15 @@ def test_job_rate_counts_every_rank():
     # 2 ranks x 4.6e9 bytes in 2.5 ms of the slowest rank
     assert bench.job_rate(2, 4.6e9, 2.5) == pytest.approx(2 * 4.6e9 / 2.5e-3)
     assert bench.job_rate(1, 1, 1000.0) == pytest.approx(1.0)
+
+
+def test_kernel_key_ignores_comments_but_not_code():
+    src = 'int a = 1;  // one\n// a comment line\n\nconst char* s = "x // y";\n'
+    assert bench._code_only(src) == 'int a = 1;\nconst char* s = "x // y";'
+    assert bench._code_only(src) != bench._code_only(src.replace("a = 1", "a = 2"))
+
+
+def test_mixed_workload_formats():
+    # QKV and O in the 2-bit + rotation format, gate+up and down ternary
+    assert [bench.product_fmt(0, mi) for mi in range(4)] == [3, 3, 1, 1]
+    assert [bench.product_fmt(2, mi) for mi in range(4)] == [2, 2, 2, 2]
