@@ -94,7 +94,11 @@ constexpr unsigned kFaultX = 4, kFaultMma = 5, kFaultDecode = 6, kFaultEpilogue 
 
 struct TcArgs {
   int64_t K, N, M;
-  const int* xexp;  // token row m of X was scaled by 2^-xexp[m]
+  const int* xexp;   // token row m of X was scaled by 2^-xexp[m]
+  const int* xflag;  // 1: row m did not convert to fp16 exactly (recomputed on CUDA cores)
+  const uint16_t* X; // the bf16 activations (for the flagged rows)
+  const uint8_t* codes;  // packed weights (for the flagged rows), group-of-four order
+  int64_t code_stride;
   uint16_t* Y;
   int tile_m;       // MMA N: tokens per tile
   int nacc;         // independent accumulators (a power of two, nacc * tile_m <= 256)
@@ -257,6 +261,71 @@ __device__ __forceinline__ void decode_quarter(const uint4 (&raw)[7], int r, uin
 // is a normal float, which is every row but those of extreme magnitude.
 __device__ __forceinline__ float scale_pow2(float v, int e) {
   return (e >= -126 && e <= 127) ? v * __int_as_float((e + 127) << 23) : ldexpf(v, e);
+}
+
+// Named barrier over `count` threads that also ORs a predicate over them: returns
+// whether any participating thread passed true.
+__device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
+// Token rows whose values span more than fp16 holds exactly after one power-of-two
+// scaling (bf16 keeps fp32's exponent range: a row may hold 2^40 next to 1.0) are
+// flagged by the conversion kernel; for them the tile's outputs are recomputed here
+// from the bf16 activations in fp32 on the CUDA cores, block by block as the pages
+// define the product (sum of +-x per block, times the block's scale). Called by all
+// kDecoders decoder threads (d = 0 .. kDecoders - 1) with the tile's flags in shared
+// memory (xf, tile_m entries) and 4 * kTileN floats of shared scratch (red); the
+// control flow depends on shared data only, so every thread meets every barrier.
+// Each flagged token's 128 outputs go to `put(t, row, value)` on threads d < kTileN.
+template <typename Put>
+__device__ __forceinline__ void fixup_flagged(const TcArgs& a, int64_t n0, int64_t m0, int kb0,
+                                              int nkb, const int* xf, float* red, int d,
+                                              Put put) {
+  const int row = d & (kTileN - 1), qtr = d / kTileN;  // 4 threads a row, blocks dealt round-robin
+  const int64_t n = n0 + row;
+  for (int t = 0; t < a.tile_m; ++t) {
+    if (!xf[t]) continue;  // shared, so uniform across the threads
+    const int64_t m = m0 + t;
+    const uint16_t* x = a.X + m * a.K;
+    float acc = 0.0f;
+    if (n < a.N) {
+      for (int kb = kb0 + qtr; kb < kb0 + nkb; kb += 4) {
+        uint32_t w[7];
+#pragma unroll
+        for (int i = 0; i < 7; ++i)
+          w[i] = __ldg(reinterpret_cast<const uint32_t*>(a.codes + g4_word_byte(n, 7 * kb + i, a.code_stride)));
+        const float s = f16_bits_to_f32(static_cast<uint16_t>(w[6] >> 16));
+        const uint16_t* xb = x + static_cast<int64_t>(kb) * kTernBlock;
+        float part = 0.0f;
+        for (int j = 0; j < kTernCodeBytes; ++j) {
+          uint32_t v = (w[j >> 2] >> (8 * (j & 3))) & 0xffu;
+          for (int i = 0; i < 5 && 5 * j + i < kTernBlock; ++i) {
+            const uint32_t dgt = v % 3u;  // digit = trit + 1
+            v /= 3u;
+            const float xv = bf16_bits_to_f32(xb[5 * j + i]);
+            if (dgt == 2u) part += xv;
+            else if (dgt == 0u) part -= xv;
+          }
+        }
+        acc += s * part;
+      }
+    }
+    red[qtr * kTileN + row] = acc;
+    named_bar_sync(3, kDecoders);
+    if (d < kTileN && n < a.N)
+      put(t, row, ((red[row] + red[kTileN + row]) + red[2 * kTileN + row]) + red[3 * kTileN + row]);
+    named_bar_sync(3, kDecoders);
+  }
 }
 
 __global__ void __launch_bounds__(kThreadsTC, 1)
@@ -495,9 +564,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       // exponents first go to shared memory (below the table, where slab 0 was)
       const uint32_t ot = tab + kHighB;
       int* xe = reinterpret_cast<int*>(smem_raw + (bstage0 - sraw));
-      for (int t = tid - 128; t < a.tile_m; t += kDecoders)
+      int* xf = xe + kMaxTileM;  // the tokens' flags (rows recomputed on the CUDA cores)
+      bool flagged = false;
+      for (int t = tid - 128; t < a.tile_m; t += kDecoders) {
         xe[t] = m0 + t < a.M ? a.xexp[m0 + t] : 0;
-      named_bar_sync(3, kDecoders);
+        xf[t] = m0 + t < a.M ? a.xflag[m0 + t] : 0;
+        flagged = flagged || xf[t] != 0;
+      }
+      flagged = named_bar_or(3, kDecoders, flagged);  // any flagged token in this tile
       const int rloc = 32 * q + lane;
       for (int c0 = 16 * grp; c0 < a.tile_m; c0 += 64) {
         uint32_t v[16];
@@ -543,6 +617,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(h[i]) : "memory");
         }
       }
+      // flagged tokens: their staged outputs are replaced by the exact recomputation
+      if (flagged) {
+        named_bar_sync(3, kDecoders);
+        fixup_flagged(a, n0, m0, kb0, nkb, xf, reinterpret_cast<float*>(xf + kMaxTileM), tid - 128,
+                      [&](int t, int rrow, float v) {
+                        const uint32_t addr = ot + static_cast<uint32_t>(t * 256 + rrow * 2);
+                        asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(f32_to_bf16_bits(v)) : "memory");
+                      });
+      }
       fence_proxy_async_smem();  // the generic-proxy writes, before the TMA reads them
       named_bar_sync(3, kDecoders);
       if (tid == 128 && ok) {
@@ -551,6 +634,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         bulk_wait_group_read0();
       }
     } else {
+      // the tile's flagged tokens (flags and scratch in the free activation slab 0)
+      int* xf = reinterpret_cast<int*>(smem_raw + (bstage0 - sraw));
+      bool flagged = false;
+      for (int t = tid - 128; t < a.tile_m; t += kDecoders) {
+        xf[t] = m0 + t < a.M ? a.xflag[m0 + t] : 0;
+        flagged = flagged || xf[t] != 0;
+      }
+      flagged = named_bar_or(3, kDecoders, flagged);
       for (int c0 = 16 * grp; c0 < a.tile_m; c0 += 64) {
         uint32_t v[16];
         tmem_ld16(lane_base + static_cast<uint32_t>(c0), v);
@@ -566,7 +657,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int64_t m = m0 + c0 + i;
-          if (m < a.M) {
+          if (m < a.M && !(flagged && a.xflag[m])) {  // flagged tokens: written by the fixup below
             // undo the activation row's power-of-two scaling (exact)
             const float y = scale_pow2(__uint_as_float(v[i]), a.xexp[m]);
             if (a.part)
@@ -575,6 +666,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
               a.Y[m * a.N + ne] = f32_to_bf16_bits(y);
           }
         }
+      }
+      if (flagged) {
+        named_bar_sync(3, kDecoders);
+        fixup_flagged(a, n0, m0, kb0, nkb, xf, reinterpret_cast<float*>(xf + kMaxTileM), tid - 128,
+                      [&](int t, int rrow, float v) {
+                        if (!ok) return;
+                        const int64_t m = m0 + t, n = n0 + rrow;
+                        if (a.part)
+                          a.part[(static_cast<int64_t>(blockIdx.z) * a.M + m) * a.N + n] = v;
+                        else
+                          a.Y[m * a.N + n] = f32_to_bf16_bits(v);
+                      });
       }
     }
   }
@@ -590,9 +693,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 // Activations to fp16, one row per CTA: x' = x * 2^-e with e chosen so that max|x'|
 // lies in [2^14, 2^15) (an exact power-of-two scaling, up or down, so rows of large
 // and of tiny activations both use fp16's full precision), rounded to nearest fp16.
+// A bf16 value lands in fp16 exactly unless it sits more than about 2^31 below the
+// row's largest (fp16's subnormal step is then coarser than its last bit); a row with
+// any such value is flagged (xflag[m] = 1) and the product recomputes its outputs
+// on the CUDA cores, so every row meets the same bound whatever its spread.
 __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t* __restrict__ X, int64_t K,
                                                         uint16_t* __restrict__ Xh,
-                                                        int* __restrict__ xexp) {
+                                                        int* __restrict__ xexp,
+                                                        int* __restrict__ xflag) {
   __shared__ float red[8];
   const int64_t m = blockIdx.x;
   // 16-byte accesses: 8 values a thread (K is a multiple of 128, rows 16-byte aligned)
@@ -618,9 +726,12 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t* __restric
   // x * 2^-e to fp16: a multiply by the power of two when it is a normal float (exact,
   // as ldexpf), ldexpf otherwise
   // (two loops: a select per element had the compiler evaluate ldexpf every time)
-  auto pack = [](float a0, float a1) {
-    return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(a0))) |
-           (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(a1))) << 16);
+  // (an inexact conversion sets `inexact`: the value does not come back from fp16)
+  bool inexact = false;
+  auto pack = [&inexact](float a0, float a1) {
+    const __half h0 = __float2half_rn(a0), h1 = __float2half_rn(a1);
+    inexact = inexact || __half2float(h0) != a0 || __half2float(h1) != a1;
+    return static_cast<uint32_t>(__half_as_ushort(h0)) | (static_cast<uint32_t>(__half_as_ushort(h1)) << 16);
   };
   if (-e >= -126 && -e <= 127) {
     const float f = __int_as_float((127 - e) << 23);
@@ -637,7 +748,11 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t* __restric
                          pack(sc(lo(v.z)), sc(hi(v.z))), pack(sc(lo(v.w)), sc(hi(v.w))));
     }
   }
-  if (threadIdx.x == 0) xexp[m] = e;
+  const int any = __syncthreads_or(inexact ? 1 : 0);
+  if (threadIdx.x == 0) {
+    xexp[m] = e;
+    xflag[m] = any ? 1 : 0;
+  }
 }
 
 // Y = bf16(sum over splits of the fp32 partial products), splits in order.
@@ -704,30 +819,33 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 }  // namespace
 
 // Workspace of the ternary tensor-core product:
-// [64 KB reserved][fp16 X: M*K][exponents: M][fp32 partials: splits*M*N when split].
+// [64 KB reserved][fp16 X: M*K][exponents: M][flags: M][fp32 partials: splits*M*N when split].
 size_t lbq_gemm_tc_workspace(const lbq_weights* w, int64_t M) {
   const TcPlan p = plan_for(w, M);
   size_t n = kWsCounterBytes + align_up(static_cast<size_t>(M) * w->K * 2, 1024) +
-             align_up(static_cast<size_t>(M) * sizeof(int), 256);
+             2 * align_up(static_cast<size_t>(M) * sizeof(int), 256);
   if (p.splits > 1) n += static_cast<size_t>(p.splits) * M * w->N * sizeof(float);
   return n;
 }
 
 cudaError_t lbq_launch_gemm_tc(const lbq_weights* w, const uint16_t* X, int64_t M, uint16_t* Y,
                                void* ws, cudaStream_t s) {
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tern_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemTC));
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  static PerDevice<bool> configured;  // the kernel's shared-memory limit, set once per device
+  bool done = false;
+  cudaError_t ce = configured.get(
+      [](int, bool* v) {
+        *v = true;
+        return cudaFuncSetAttribute(gemm_tern_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(kSmemTC));
+      },
+      &done);
+  if (ce != cudaSuccess) return ce;
   char* base = static_cast<char*>(ws) + kWsCounterBytes;
   uint16_t* Xh = reinterpret_cast<uint16_t*>(base);
   int* xexp = reinterpret_cast<int*>(base + align_up(static_cast<size_t>(M) * w->K * 2, 1024));
-  x_to_f16_kernel<<<static_cast<unsigned>(M), 256, 0, s>>>(X, w->K, Xh, xexp);
+  int* xflag = reinterpret_cast<int*>(reinterpret_cast<char*>(xexp) +
+                                      align_up(static_cast<size_t>(M) * sizeof(int), 256));
+  x_to_f16_kernel<<<static_cast<unsigned>(M), 256, 0, s>>>(X, w->K, Xh, xexp, xflag);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
@@ -736,6 +854,10 @@ cudaError_t lbq_launch_gemm_tc(const lbq_weights* w, const uint16_t* X, int64_t 
   a.N = w->N;
   a.M = M;
   a.xexp = xexp;
+  a.xflag = xflag;
+  a.X = X;
+  a.codes = static_cast<const uint8_t*>(w->codes);
+  a.code_stride = w->code_stride;
   a.Y = Y;
   const TcPlan plan = plan_for(w, M);
   a.tile_m = plan.tile_m;
@@ -743,7 +865,7 @@ cudaError_t lbq_launch_gemm_tc(const lbq_weights* w, const uint16_t* X, int64_t 
   while (a.nacc < 8 && 2 * a.nacc * a.tile_m <= static_cast<int>(kAccCols)) a.nacc *= 2;
   a.kb_per_split = plan.kb_per_split;
   a.part = plan.splits > 1
-               ? reinterpret_cast<float*>(reinterpret_cast<char*>(xexp) +
+               ? reinterpret_cast<float*>(reinterpret_cast<char*>(xflag) +
                                           align_up(static_cast<size_t>(M) * sizeof(int), 256))
                : nullptr;
   a.fault = lbq_fault_word();

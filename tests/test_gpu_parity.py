@@ -335,3 +335,146 @@ def test_bounded_wait_gives_up_and_device_stays_usable(L, orc):
     Y, B = orc.gemm(TERN5, codes, scales, K, synth.bf16_bits(x), None)
     _check_products(y, Y[0], B[0], "after a timed-out wait")
     assert L.lbq_device_fault() == 0
+
+
+# ------------------------------------------------------- tensor-core product: edge cases
+
+def _spread_rows(M, K, seed):
+    """bf16 activation rows that fp16 cannot hold after one power-of-two scaling, next to
+    ordinary ones: row 0 = [2^40, 1.0078125, ...], row 1 = [2^34, 1.0078125, ...], row 2 =
+    random signs and exponents over 2^-60 .. 2^60, row 3 = N(0, 1), row 4 = zeros, the
+    rest N(0, 1) with a few entries scaled by 2^-45."""
+    assert M >= 4
+    g = torch.Generator().manual_seed(seed)
+    X = torch.randn((max(M, 5), K), generator=g)
+    X[0] = 1.0078125
+    X[0, 0] = 2.0 ** 40
+    X[1] = 1.0078125
+    X[1, 0] = 2.0 ** 34
+    e = torch.randint(-60, 61, (K,), generator=g).double()
+    X[2] = (torch.sign(torch.randn(K, generator=g)) * (1 + torch.rand(K, generator=g)) * 2.0 ** e).float()
+    X[4] = 0.0
+    X = X[:M]
+    for r in range(5, M):
+        X[r, r % K] *= 2.0 ** -45
+    return X.to(torch.bfloat16)
+
+
+def _spread_weights(N, K, seed):
+    """Rows whose trit is 0 at k = 0 and +1 elsewhere (the large entry of rows 0 and 1
+    meets a zero weight), every fourth row ordinary N(0, 0.02^2) weights."""
+    W = torch.full((N, K), 0.02)
+    W[:, 0] = 0.0
+    R = synth.weights(N, K, seed)
+    W[::4] = R[::4]
+    return W
+
+
+@pytest.mark.parametrize("M,N,K", [(6, 128, 512),      # one tile, Y through one TMA store
+                                   (6, 256, 5120),     # K split over the grid: fp32 partials
+                                   (4, 130, 512),      # N * 2 not 16-aligned: direct stores
+                                   (20, 130, 1024),    # direct stores and a K split
+                                   (300, 1000, 2048)]) # two token tiles
+def test_ternary_gemm_rows_wider_than_fp16(L, orc, M, N, K):
+    """Activation rows whose values span more than fp16 holds after a power-of-two scaling
+    (2^40 beside 1.0078125, exponents over +-60) meet the bound like any other row."""
+    W = _spread_weights(N, K, 8100 + N)
+    X = _spread_rows(M, K, 8200 + M)
+    pw, codes, scales = _pack_both(L, orc, TERN5, W)
+    Yg = L.lbq_gemm(pw, X.cuda())
+    Y, B = orc.gemm(TERN5, codes, scales, K, synth.bf16_bits(X), None, nthreads=NTHREADS)
+    _check_products(Yg, Y, B, f"wide rows M={M} N={N} K={K}")
+    assert L.lbq_device_fault() == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(8, 1, 512), (16, 129, 640), (5, 4 * 33 + 1, 1024)])
+def test_ternary_gemm_tensor_core_ragged_n(L, orc, M, N, K):
+    W = synth.weights(N, K, 8300 + N)
+    X = synth.activations(M, K, 8400 + M)
+    pw, codes, scales = _pack_both(L, orc, TERN5, W)
+    Yg = L.lbq_gemm(pw, X.cuda())
+    Y, B = orc.gemm(TERN5, codes, scales, K, synth.bf16_bits(X), None, nthreads=NTHREADS)
+    _check_products(Yg, Y, B, f"ragged N={N} M={M}")
+
+
+@pytest.mark.parametrize("M", (8, 64))
+def test_ternary_gemm_zero_blocks_give_exact_zero(L, M):
+    """An all-zero weight block contributes exactly nothing on the tensor cores too: rows
+    whose every block is zero give exactly 0, and a zero activation matrix gives 0."""
+    N, K = 256, 1024
+    W = synth.weights(N, K, 8500)
+    W[7:13] = 0.0
+    W[100, 128:256] = 0.0   # one zero block in an otherwise ordinary row
+    pw = L.lbq_pack(TERN5, W.cuda())
+    X = synth.activations(M, K, 8600).cuda()
+    Y = L.lbq_gemm(pw, X).float().cpu()
+    assert torch.all(Y[:, 7:13] == 0)
+    Y0 = L.lbq_gemm(pw, torch.zeros((M, K), dtype=torch.bfloat16, device="cuda"))
+    assert torch.all(Y0.float() == 0)
+
+
+@pytest.mark.parametrize("mi", (0, 3))
+def test_ternary_gemm_m4096_27b_sampled(L, orc, mi):
+    """M = 4096 tokens through the 27B QKV (K = 5120) and down (K = 17408) products, the
+    bench's largest batch; sampled weight rows checked over every token."""
+    name, K, N = synth.LAYER_SHAPES[mi]
+    M = 4096
+    Wd = synth.weights(N, K, 9900 + mi, device="cuda")
+    pw = L.lbq_pack(TERN5, Wd)
+    X = synth.activations(M, K, 9950 + mi, device="cuda")
+    Yg = L.lbq_gemm(pw, X)
+    rows = torch.tensor([0, 1, 2, 3, 127, 128, 2049, N - 130, N - 1], device="cuda")
+    codes, scales = orc.pack(TERN5, Wd[rows].cpu().numpy())
+    Y, B = orc.gemm(TERN5, codes, scales, K, synth.bf16_bits(X), None, nthreads=NTHREADS)
+    _check_products(Yg[:, rows], Y, B, f"27B {name}, M=4096")
+
+
+# ------------------------------------------------------- mixed-format layer, one graph
+
+def test_mixed_format_layer_graph_chained(L, orc):
+    """One 27B-shaped layer with 2-bit + rotation attention (QKV, O) and ternary FFN
+    (gate+up, down), captured in one CUDA graph as the bench's mixed pass runs it: every
+    product chained to the previous kernel by programmatic dependent launch. Gate+up
+    reads the O product's output as its input, so a product that read its x before the
+    previous kernel finished would see stale values; O's input is changed between
+    replays to make such a read visible. Every output is checked against the oracle."""
+    fmts = (Q2RHT, Q2RHT, TERN5, TERN5)
+    prods = []
+    for mi, (name, K, N) in enumerate(synth.LAYER_SHAPES):
+        Wd = synth.weights(N, K, synth.seed_of(40, 0, mi), device="cuda")
+        pw = L.lbq_pack(fmts[mi], Wd)
+        codes, scales = orc.pack(fmts[mi], Wd.cpu().numpy())
+        del Wd
+        x = synth.activations(1, K, synth.seed_of(50, 0, mi), device="cuda")[0].clone()
+        prods.append(dict(name=name, K=K, N=N, fmt=fmts[mi], pw=pw, codes=codes, scales=scales,
+                          x=x, y=torch.empty(N, dtype=torch.bfloat16, device="cuda")))
+    prods[2]["x"] = prods[1]["y"]  # gate+up reads O's output
+    Dg = {K: L.lbq_rht_signs(31 + K, K) for K in (synth.HIDDEN, synth.FFN)}
+    Do = {K: orc.rht_signs(31 + K, K) for K in (synth.HIDDEN, synth.FFN)}
+    ws = torch.zeros(max(L.lbq_workspace_bytes(p["pw"], 1) for p in prods), dtype=torch.uint8,
+                     device="cuda")
+    stream = torch.cuda.Stream()
+
+    def step():
+        for p in prods:
+            L.lbq_gemv(p["pw"], p["x"], Dg[p["K"]] if p["fmt"] == Q2RHT else None, p["y"], ws,
+                       stream=stream)
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        step()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            step()
+    x_o = prods[1]["x"]
+    for rep in range(3):
+        with torch.cuda.stream(stream):
+            x_o.copy_(synth.activations(1, synth.HIDDEN, 60 + rep, device="cuda")[0])
+            g.replay()
+        torch.cuda.synchronize()
+        for p in prods:
+            Xb = synth.bf16_bits(p["x"].view(1, -1))
+            Y, B = orc.gemm(p["fmt"], p["codes"], p["scales"], p["K"], Xb,
+                            Do[p["K"]] if p["fmt"] == Q2RHT else None, nthreads=NTHREADS)
+            _check_products(p["y"], Y[0], B[0], f"mixed {p['name']} replay {rep}")
+    assert L.lbq_device_fault() == 0
