@@ -12,7 +12,7 @@ inline bool aligned(const void* p, uintptr_t a) {
 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
-inline lbq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LBQ_OK : LBQ_ERR_CUDA; }
+inline lbq_status from_cuda(cudaError_t e) { return lbq_cuda_status(e); }
 
 // Up to kTernPerTokenMaxM tokens a ternary product runs as one batch-1 product per
 // token: on the tensor cores a 16-token tile costs about as much as a 2-token one
@@ -50,8 +50,9 @@ lbq_status check_weights(const lbq_weights* w, Layout* L) {
   return LBQ_OK;
 }
 
-lbq_status check_product(const lbq_weights* w, const void* x, int64_t M, const int8_t* D,
-                         const void* y, void* ws, size_t ws_bytes, Layout* L) {
+// Every check of a product call but the workspace's.
+lbq_status check_operands(const lbq_weights* w, const void* x, int64_t M, const int8_t* D,
+                          const void* y, Layout* L) {
   lbq_status st = check_weights(w, L);
   if (st != LBQ_OK) return st;
   if (M < 1) return LBQ_ERR_SHAPE;
@@ -61,6 +62,14 @@ lbq_status check_product(const lbq_weights* w, const void* x, int64_t M, const i
     if (!D) return LBQ_ERR_ARG;
     if (!aligned(D, 16)) return LBQ_ERR_ALIGN;
   }
+  if (M == 1 && lbq_gemv_workspace(w) && w->N > lbq::kMaxSplitRows) return LBQ_ERR_SHAPE;
+  return LBQ_OK;
+}
+
+lbq_status check_product(const lbq_weights* w, const void* x, int64_t M, const int8_t* D,
+                         const void* y, void* ws, size_t ws_bytes, Layout* L) {
+  lbq_status st = check_operands(w, x, M, D, y, L);
+  if (st != LBQ_OK) return st;
   const size_t need = lbq_workspace_bytes(w, M);
   if (need) {
     if (!ws || ws_bytes < need) return LBQ_ERR_WORKSPACE;
@@ -71,7 +80,69 @@ lbq_status check_product(const lbq_weights* w, const void* x, int64_t M, const i
 
 }  // namespace
 
+lbq_status lbq_validate_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D,
+                             const uint16_t* y) {
+  Layout L;
+  return check_operands(w, x, 1, D, y, &L);
+}
+
+namespace {
+
+// Byte ranges [lo, hi) overlap.
+inline bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// A batch list: every product valid on its own (as for lbq_gemv, without its limit on
+// split rows, which the batch kernel does not have), and no output overlapping an
+// input or another output.
+lbq_status check_batch(const lbq_product* ps, int32_t n) {
+  if (!ps || n < 1) return LBQ_ERR_ARG;
+  for (int32_t i = 0; i < n; ++i) {
+    Layout L;
+    const lbq_weights* w = &ps[i].w;
+    lbq_status st = check_weights(w, &L);
+    if (st != LBQ_OK) return st;
+    if (w->N > (int64_t{1} << 28)) return LBQ_ERR_SHAPE;
+    if (!ps[i].x || !ps[i].y) return LBQ_ERR_ARG;
+    if (!aligned(ps[i].x, 16) || !aligned(ps[i].y, 2)) return LBQ_ERR_ALIGN;
+    if (w->fmt == LBQ_Q2RHT) {
+      if (!ps[i].D) return LBQ_ERR_ARG;
+      if (!aligned(ps[i].D, 16)) return LBQ_ERR_ALIGN;
+    }
+  }
+  for (int32_t i = 0; i < n; ++i) {
+    const size_t ny = static_cast<size_t>(ps[i].w.N) * 2;
+    for (int32_t k = 0; k < n; ++k) {
+      const size_t nx = static_cast<size_t>(ps[k].w.K) * 2;
+      if (overlap(ps[i].y, ny, ps[k].x, nx)) return LBQ_ERR_ARG;
+      if (ps[k].D && overlap(ps[i].y, ny, ps[k].D, static_cast<size_t>(ps[k].w.K))) return LBQ_ERR_ARG;
+      if (k != i && overlap(ps[i].y, ny, ps[k].y, static_cast<size_t>(ps[k].w.N) * 2)) return LBQ_ERR_ARG;
+    }
+  }
+  return LBQ_OK;
+}
+
+}  // namespace
+
+namespace {
+thread_local int g_last_cuda_error = 0;
+}  // namespace
+
+lbq_status lbq_cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return LBQ_OK;
+  g_last_cuda_error = static_cast<int>(e);
+  return LBQ_ERR_CUDA;
+}
+
 extern "C" {
+
+int32_t lbq_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* lbq_last_cuda_error_string(void) {
+  return g_last_cuda_error ? cudaGetErrorString(static_cast<cudaError_t>(g_last_cuda_error)) : "no error";
+}
 
 const char* lbq_status_string(lbq_status st) {
   switch (st) {
@@ -143,10 +214,11 @@ lbq_status lbq_hadamard(const uint16_t* x, const int8_t* D, int64_t M, int64_t K
 lbq_status lbq_device_fault(uint32_t* code) {
   if (!code) return LBQ_ERR_ARG;
   unsigned* word = lbq_fault_word();
-  if (!word) return LBQ_ERR_CUDA;
+  if (!word) return lbq_cuda_status(cudaErrorInvalidDevicePointer);
   unsigned v = 0;
-  if (cudaMemcpy(&v, word, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return LBQ_ERR_CUDA;
-  if (v && cudaMemset(word, 0, sizeof(v)) != cudaSuccess) return LBQ_ERR_CUDA;
+  cudaError_t e = cudaMemcpy(&v, word, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return lbq_cuda_status(e);
+  if (v && (e = cudaMemset(word, 0, sizeof(v))) != cudaSuccess) return lbq_cuda_status(e);
   *code = v;
   return v ? LBQ_ERR_DEVICE_WAIT : LBQ_OK;
 }
@@ -164,8 +236,35 @@ lbq_status lbq_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D, ui
   Layout L;
   lbq_status st = check_product(w, x, 1, D, y, workspace, workspace_bytes, &L);
   if (st != LBQ_OK) return st;
-  if (lbq_gemv_workspace(w) && w->N > lbq::kMaxSplitRows) return LBQ_ERR_SHAPE;
   return from_cuda(lbq_launch_gemv(w, x, D, y, workspace, as_stream(stream)));
+}
+
+size_t lbq_gemv_batch_workspace_bytes(const lbq_product* ps, int32_t n) {
+  if (check_batch(ps, n) != LBQ_OK) return 0;
+  size_t need = 0;
+  for (int32_t i = 0; i < n; i += LBQ_BATCH_MAX) {
+    const size_t b = lbq_gemv_batch_ws(ps + i, n - i < LBQ_BATCH_MAX ? n - i : LBQ_BATCH_MAX);
+    if (b > need) need = b;
+  }
+  return need;
+}
+
+lbq_status lbq_gemv_batch(const lbq_product* ps, int32_t n, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  lbq_status st = check_batch(ps, n);
+  if (st != LBQ_OK) return st;
+  const size_t need = lbq_gemv_batch_workspace_bytes(ps, n);
+  if (!workspace || workspace_bytes < need) return LBQ_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return LBQ_ERR_ALIGN;
+  for (int32_t i = 0; i < n; i += LBQ_BATCH_MAX) {
+    const cudaError_t e = lbq_launch_gemv_batch(ps + i, n - i < LBQ_BATCH_MAX ? n - i : LBQ_BATCH_MAX,
+                                                workspace, as_stream(stream));
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return lbq_cuda_status(e);
+    }
+  }
+  return LBQ_OK;
 }
 
 lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const int8_t* D,
@@ -179,7 +278,7 @@ lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const in
     for (int64_t m = 0; m < M; ++m) {
       const cudaError_t e =
           lbq_launch_gemv(w, X + m * w->K, D, Y + m * w->N, workspace, as_stream(stream));
-      if (e != cudaSuccess) return LBQ_ERR_CUDA;
+      if (e != cudaSuccess) return lbq_cuda_status(e);
     }
     return LBQ_OK;
   }

@@ -49,19 +49,19 @@
 //    before this one starts. x, y and the workspace are touched only after the wait.
 #include <type_traits>
 
-#include "rht.cuh"
+#include "lut.cuh"
 #include "sm100_async.cuh"
 
 namespace {
 
 using namespace lbq;
+using namespace lbq::lut;
 
 constexpr int kWarps = 16;                    // consumer warps
 constexpr int kThreads = 32 * kWarps;         // consumer threads
 constexpr int kBlockThreads = kThreads + 32;  // + the copy-issuing warp
 constexpr int kRows = 16;                     // rows per unit (four groups of four)
 constexpr int kSub = 4;                       // units per ring slot (one tensor copy)
-constexpr uint32_t kPage = 65536;             // table page: 256 values x 256 bytes
 // Shared memory: the 128 KB table at the first 64 KB boundary of the window (its
 // page addressing keeps the base in the upper half of the PRMT operand); below it
 // (the dynamic window starts 1 KB into shared memory on sm_100) the x slice, the
@@ -77,56 +77,11 @@ constexpr uint32_t kMisc = (kXBytes + 2 * 8 * kMaxSlots + 8 + 1023) & ~1023u;
 constexpr uint32_t kSmem = 225 * 1024;
 constexpr unsigned kFaultLayout = 3, kFaultRing = 10;
 
+using lut::Traits;
+using lut::kPage;
+// A ring slot: kSub 16-row units of a slice, codes first, then scales.
 template <int FMT>
-struct Traits;
-// kGroupBytes: a group of four rows' codes in one slice; kScaleBytes: its scales
-// (1-bit and 2-bit; ternary scales sit among the codes); kSlot: a ring slot of kSub
-// 16-row units, codes first, then scales.
-template <>
-struct Traits<LBQ_TERN5> {
-  static constexpr int kWeights = 512, kWords = 28, kBlocks = 4, kDigits = 5;
-  static constexpr uint32_t kGroupBytes = 16 * kWords, kScaleBytes = 0;
-  static constexpr uint32_t kSlot = 4 * kSub * (kGroupBytes + kScaleBytes);
-};
-template <>
-struct Traits<LBQ_SIGN1> {
-  static constexpr int kWeights = 1024, kWords = 32, kBlocks = 8, kDigits = 8;
-  static constexpr uint32_t kGroupBytes = 16 * kWords, kScaleBytes = 8 * kBlocks;
-  static constexpr uint32_t kSlot = 4 * kSub * (kGroupBytes + kScaleBytes);
-};
-template <>
-struct Traits<LBQ_Q2RHT> {
-  static constexpr int kWeights = 512, kWords = 32, kBlocks = 16, kDigits = 4;
-  static constexpr uint32_t kGroupBytes = 16 * kWords, kScaleBytes = 8 * kBlocks;
-  static constexpr uint32_t kSlot = 4 * kSub * (kGroupBytes + kScaleBytes);
-};
-
-// Word of the slice that lane l handles (ternary: block l/8, word l%8 of it; lanes
-// 7, 15, 23, 31 have none), or -1; nb = blocks present in this slice.
-template <int FMT>
-__device__ __forceinline__ int lane_word(int l, int nb) {
-  if (FMT == LBQ_TERN5) return ((l & 7) < 7 && (l >> 3) < nb) ? 7 * (l >> 3) + (l & 7) : -1;
-  if (FMT == LBQ_SIGN1) return l < 4 * nb ? l : -1;
-  return l;
-}
-
-// Weight index (within the slice) of digit e of byte `slot` of lane l's word, or -1
-// if that digit carries no weight (scale bytes, byte-25 padding digits, no word).
-template <int FMT>
-__device__ __forceinline__ int digit_weight(int slot, int l, int e, int nb) {
-  const int w = lane_word<FMT>(l, nb);
-  if (w < 0) return -1;
-  if (FMT == LBQ_TERN5) {
-    const int bb = w / 7, c = 4 * (w % 7) + slot;  // byte within the 28-byte block
-    if (c >= kTernCodeBytes) return -1;            // the block's fp16 scale
-    const int kb = 5 * c + e;
-    return kb < kTernBlock ? bb * kTernBlock + kb : -1;
-  } else if (FMT == LBQ_SIGN1) {
-    return 32 * w + 8 * slot + e;
-  } else {
-    return 16 * w + 4 * slot + e;
-  }
-}
+constexpr uint32_t kSlotBytes = 4 * kSub * (Traits<FMT>::kGroupBytes + Traits<FMT>::kScaleBytes);
 
 template <int FMT>
 // The packed weights reach the kernel as tensor maps (see the launch).
@@ -142,198 +97,6 @@ struct Args {
   unsigned* fault;  // the device fault word (layout check, bounded waits)
 };
 
-__device__ __forceinline__ void sts_f2(uint32_t addr, float2 v) {
-  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(v.x), "f"(v.y) : "memory");
-}
-template <uint32_t kImm>
-__device__ __forceinline__ float lds_imm(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(kImm));
-  return v;
-}
-__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ uint2 lds_v2(uint32_t addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ float2 h2_to_f2(uint32_t h2) {
-  return __half22float2(*reinterpret_cast<const __half2*>(&h2));
-}
-
-// Table entries of one row word: the four bytes' partial sums added up.
-// Slot i lives on page i/2 at column offset (i%2)*128; `lanereg` = table base | lane*4.
-__device__ __forceinline__ float2 lookup_pair(uint32_t w0, uint32_t w1, uint32_t lanereg) {
-  const float2 e0 = make_float2(lds_imm<0>(__byte_perm(w0, lanereg, 0x7604)),
-                                lds_imm<0>(__byte_perm(w1, lanereg, 0x7604)));
-  const float2 e1 = make_float2(lds_imm<128>(__byte_perm(w0, lanereg, 0x7614)),
-                                lds_imm<128>(__byte_perm(w1, lanereg, 0x7614)));
-  const float2 e2 = make_float2(lds_imm<kPage>(__byte_perm(w0, lanereg, 0x7624)),
-                                lds_imm<kPage>(__byte_perm(w1, lanereg, 0x7624)));
-  const float2 e3 = make_float2(lds_imm<kPage + 128>(__byte_perm(w0, lanereg, 0x7634)),
-                                lds_imm<kPage + 128>(__byte_perm(w1, lanereg, 0x7634)));
-  return __fadd2_rn(__fadd2_rn(e0, e1), __fadd2_rn(e2, e3));
-}
-
-// The x slice of slice j, loaded by x_issue (plain loads: the weights come through
-// the copy engine, whose queue would hold x back behind them) and stored to shared
-// memory as fp32 by x_store.
-struct XLoad {
-  uint4 v0, v1, d;
-};
-template <int FMT>
-__device__ __forceinline__ XLoad x_issue(const Args<FMT>& a, int32_t j, int tid) {
-  using T = Traits<FMT>;
-  XLoad r{make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
-  const int64_t k0 = static_cast<int64_t>(j) * T::kWeights;
-  if (FMT == LBQ_Q2RHT) {
-    if (tid < 32) {  // one warp: 16 activations and 16 signs per lane
-      const uint4* x4 = reinterpret_cast<const uint4*>(a.x + k0 + 16 * tid);
-      r.v0 = x4[0];
-      r.v1 = x4[1];
-      r.d = *reinterpret_cast<const uint4*>(a.D + k0 + 16 * tid);
-    }
-  } else {
-    const int blk0 = j * T::kBlocks;
-    const int nb = a.nblk - blk0 < T::kBlocks ? a.nblk - blk0 : T::kBlocks;
-    // one 16-byte load of 8 activations per thread (x and the slices are 16-byte aligned)
-    if (tid < T::kWeights / 8 && 8 * tid < nb * kTernBlock)
-      r.v0 = __ldg(reinterpret_cast<const uint4*>(a.x + k0) + tid);
-  }
-  return r;
-}
-template <int FMT>
-__device__ __forceinline__ void x_store(const XLoad& r, float* xs, int tid) {
-  using T = Traits<FMT>;
-  if (FMT == LBQ_Q2RHT) {
-    if (tid < 32) {
-      const uint32_t xw[8] = {r.v0.x, r.v0.y, r.v0.z, r.v0.w, r.v1.x, r.v1.y, r.v1.z, r.v1.w};
-      const uint32_t dw[4] = {r.d.x, r.d.y, r.d.z, r.d.w};
-      float v[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint32_t bits = (i & 1) ? (xw[i >> 1] & 0xffff0000u) : (xw[i >> 1] << 16);
-        const int8_t sgn = static_cast<int8_t>((dw[i >> 2] >> (8 * (i & 3))) & 0xff);
-        const float xv = __uint_as_float(bits);
-        v[i] = sgn < 0 ? -xv : xv;
-      }
-      fwht512_warp(v);
-      float4* d = reinterpret_cast<float4*>(xs + 16 * tid);
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        d[q] = make_float4(v[4 * q] * kRhtNorm, v[4 * q + 1] * kRhtNorm, v[4 * q + 2] * kRhtNorm,
-                           v[4 * q + 3] * kRhtNorm);
-    }
-  } else if (tid < T::kWeights / 8) {
-    const uint32_t w[4] = {r.v0.x, r.v0.y, r.v0.z, r.v0.w};
-    float f[8];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      f[2 * q] = __uint_as_float(w[q] << 16);
-      f[2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
-    }
-    float4* d = reinterpret_cast<float4*>(xs + 8 * tid);
-    d[0] = make_float4(f[0], f[1], f[2], f[3]);
-    d[1] = make_float4(f[4], f[5], f[6], f[7]);
-  }
-}
-
-// Builds the lookup table for slice j from the x slice in shared memory (all threads).
-// Thread t owns table column pair t % 64 (lanes 2c, 2c+1 of one byte slot) and the
-// values v = lo + R * hi for hi = t / 64, t / 64 + 8, ...; everything that does not
-// depend on hi is computed once.
-template <int FMT>
-__device__ __forceinline__ void build_table(const Args<FMT>& a, int32_t j, uint32_t tbase,
-                                            const float* xs, int tid) {
-  using T = Traits<FMT>;
-  const int blk0 = j * T::kBlocks;
-  const int nb = a.nblk - blk0 < T::kBlocks ? a.nblk - blk0 : T::kBlocks;
-  const int cp = tid & 63;
-  const int slot = cp >> 4, l0 = 2 * (cp & 15);
-  float2 xv[T::kDigits];
-#pragma unroll
-  for (int e = 0; e < T::kDigits; ++e) {
-    const int ka = digit_weight<FMT>(slot, l0, e, nb);
-    const int kb = digit_weight<FMT>(slot, l0 + 1, e, nb);
-    xv[e] = make_float2(ka >= 0 ? xs[ka] : 0.0f, kb >= 0 ? xs[kb] : 0.0f);
-  }
-  const uint32_t col = tbase + (slot >> 1) * kPage + (slot & 1) * 128 + l0 * 4;
-  constexpr int kStep = kThreads / 64;
-  if (FMT == LBQ_TERN5) {
-    // v = d0 + 3 d1 + 9 d2 + 27 (d3 + 3 d4); entry = sum_e (d_e - 1) x_e
-    float2 ab[9];
-#pragma unroll
-    for (int m = 0; m < 9; ++m) {
-      const float l0f = static_cast<float>(m % 3 - 1), l1f = static_cast<float>(m / 3 - 1);
-      ab[m] = __ffma2_rn(make_float2(l0f, l0f), xv[0], __fmul2_rn(make_float2(l1f, l1f), xv[1]));
-    }
-    // 27 runs of 9 values (digits 2..4 fixed) per column pair, dealt round-robin:
-    // at most 4 runs a thread
-    for (int hd = tid >> 6; hd < 27; hd += kStep) {
-      const int hi = hd / 3, d2 = hd - 3 * hi;
-      const float l3 = static_cast<float>(hi % 3 - 1), l4 = static_cast<float>(hi / 3 - 1);
-      const float2 q = __ffma2_rn(make_float2(l3, l3), xv[3], __fmul2_rn(make_float2(l4, l4), xv[4]));
-      const float l = static_cast<float>(d2 - 1);
-      const float2 qc = __ffma2_rn(make_float2(l, l), xv[2], q);
-      const uint32_t row0 = col + static_cast<uint32_t>(9 * d2 + 27 * hi) * 256u;
-#pragma unroll
-      for (int m = 0; m < 9; ++m) sts_f2(row0 + m * 256u, __fadd2_rn(qc, ab[m]));
-    }
-    // byte values 243..255 never occur: zero rows keep them harmless
-    for (int i = tid; i < 13 * 64; i += kThreads) {
-      const int v = 243 + i / 64, c = i % 64;
-      sts_f2(tbase + (c >> 5) * kPage + static_cast<uint32_t>(v) * 256u + (c & 31) * 8,
-             make_float2(0.0f, 0.0f));
-    }
-  } else {
-    // v = lo + 16 hi; the low two digits come from lo & 3 and lo >> 2
-    float2 av[4], bv[4];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      if (FMT == LBQ_SIGN1) {
-        const float s0 = (m & 1) ? 1.0f : -1.0f, s1 = (m & 2) ? 1.0f : -1.0f;
-        av[m] = __ffma2_rn(make_float2(s0, s0), xv[0], __fmul2_rn(make_float2(s1, s1), xv[1]));
-        bv[m] = __ffma2_rn(make_float2(s0, s0), xv[2], __fmul2_rn(make_float2(s1, s1), xv[3]));
-      } else {
-        const float l = static_cast<float>(m) - 1.5f;
-        av[m] = __fmul2_rn(make_float2(l, l), xv[0]);
-        bv[m] = __fmul2_rn(make_float2(l, l), xv[1]);
-      }
-    }
-    for (int hi = tid >> 6; hi < 16; hi += kStep) {
-      float2 q;
-      if (FMT == LBQ_SIGN1) {
-        q = make_float2(0.0f, 0.0f);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float l = ((hi >> e) & 1) ? 1.0f : -1.0f;
-          q = __ffma2_rn(make_float2(l, l), xv[4 + e], q);
-        }
-      } else {
-        const float l2 = static_cast<float>(hi & 3) - 1.5f, l3 = static_cast<float>(hi >> 2) - 1.5f;
-        q = __ffma2_rn(make_float2(l2, l2), xv[2], __fmul2_rn(make_float2(l3, l3), xv[3]));
-      }
-#pragma unroll
-      for (int m1 = 0; m1 < 4; ++m1) {
-        const float2 qb = __fadd2_rn(q, bv[m1]);
-        const uint32_t row0 = col + static_cast<uint32_t>(4 * m1 + 16 * hi) * 256u;
-#pragma unroll
-        for (int m0 = 0; m0 < 4; ++m0) sts_f2(row0 + m0 * 256u, __fadd2_rn(qb, av[m0]));
-      }
-    }
-  }
-  named_bar_sync(1, kThreads);
-}
-
 // One CTA: kWarps consumer warps and one warp that issues the weight copies. At most
 // 112 registers a thread (544 x 112 = 60928 of the SM's 65536), so that a CTA of the
 // split-K sum kernel (128 threads x 32) always fits beside it. tm_c / tm_s: the
@@ -348,7 +111,7 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
   constexpr bool kSepScales = FMT != LBQ_TERN5;
   constexpr uint32_t kScaleOff = 4 * kSub * T::kGroupBytes;  // scales within a slot
   static_assert(kWarps % kSub == 0, "whole warp groups");
-  static_assert(T::kSlot % 128 == 0 && kScaleOff % 128 == 0 && (4 * T::kGroupBytes) % 128 == 0 &&
+  static_assert(kSlotBytes<FMT> % 128 == 0 && kScaleOff % 128 == 0 && (4 * T::kGroupBytes) % 128 == 0 &&
                     (4 * T::kScaleBytes) % 128 == 0,
                 "tensor copies land on 128-byte boundaries");
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -363,8 +126,8 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
   const uint32_t misc = misc_low ? sbase : ttop;
   const uint32_t lo0 = misc_low ? sbase + kMisc : sbase;  // ring slots below the table
   const uint32_t hi0 = misc_low ? ttop : ttop + kMisc;    // ... and above it
-  const int s_lo = static_cast<int>((tbase - lo0) / T::kSlot);
-  const int s_hi = hi0 < send ? static_cast<int>((send - hi0) / T::kSlot) : 0;
+  const int s_lo = static_cast<int>((tbase - lo0) / kSlotBytes<FMT>);
+  const int s_hi = hi0 < send ? static_cast<int>((send - hi0) / kSlotBytes<FMT>) : 0;
   // The slot count is a multiple of the kWarps / kSub warp groups: unit sequence
   // number q goes to slot q % S and is taken by group q % (kWarps / kSub), so every
   // slot belongs to one group, which waits for a slot's next fill only after taking
@@ -379,8 +142,8 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
   const uint32_t full0 = misc + kXBytes, empty0 = full0 + 8 * kMaxSlots;
   const uint32_t built = empty0 + 8 * kMaxSlots;  // the table is built (inside kMisc)
   auto slot_addr = [&](int s) {
-    return s < s_lo ? lo0 + static_cast<uint32_t>(s) * T::kSlot
-                    : hi0 + static_cast<uint32_t>(s - s_lo) * T::kSlot;
+    return s < s_lo ? lo0 + static_cast<uint32_t>(s) * kSlotBytes<FMT>
+                    : hi0 + static_cast<uint32_t>(s - s_lo) * kSlotBytes<FMT>;
   };
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -470,9 +233,10 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
   }
 
   pdl_wait();  // x, y and the workspace may belong to the previous kernel until here
-  x_store<FMT>(x_issue<FMT>(a, j, tid), xs, tid);
+  x_store<FMT>(x_issue<FMT>(a.x, a.D, a.nblk, j, tid), xs, tid);
   named_bar_sync(1, kThreads);
-  build_table<FMT>(a, j, tbase, xs, tid);
+  build_table<FMT, kThreads>(nb, tbase, xs, tid);
+  named_bar_sync(1, kThreads);
   if (tid == 0) mbar_arrive(built);
 
   // This lane's word of each group, and (1-bit, 2-bit) its block's scales of four
@@ -645,16 +409,16 @@ int slices_of(const lbq_weights* w) {
 template <int FMT>
 cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uint16_t* y, void* ws,
                    cudaStream_t s) {
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_lut_kernel<FMT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmem));
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  static PerDevice<bool> configured;  // the kernel's shared-memory limit, set once per device
+  bool ok = false;
+  cudaError_t ce = configured.get(
+      [](int, bool* v) {
+        *v = true;
+        return cudaFuncSetAttribute(gemv_lut_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(kSmem));
+      },
+      &ok);
+  if (ce != cudaSuccess) return ce;
   Args<FMT> a;
   a.K = w->K;
   a.N = w->N;
@@ -741,15 +505,22 @@ cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uin
 }  // namespace
 
 unsigned* lbq_fault_word() {
-  static unsigned* addr[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_fault_word) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<unsigned*>(p);
+  static PerDevice<unsigned*> addr;  // looked up once per device, with that device current
+  unsigned* a = nullptr;
+  const cudaError_t e = addr.get(
+      [](int, unsigned** v) {
+        void* p = nullptr;
+        const cudaError_t r = cudaGetSymbolAddress(&p, g_fault_word);
+        if (r != cudaSuccess) return r;
+        *v = static_cast<unsigned*>(p);
+        return cudaSuccess;
+      },
+      &a);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
   }
-  return addr[dev];
+  return a;
 }
 
 size_t lbq_gemv_workspace(const lbq_weights* w) {

@@ -6,6 +6,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "lbq.h"
 
 namespace lbq {
@@ -87,20 +90,60 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-inline int sm_count() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-    cached[dev] = n;
+constexpr int kMaxDevices = 64;
+
+// A value computed once per device, on first use with that device current, from any
+// number of host threads: the first caller for a device runs `make` under a lock; a
+// failed `make` is retried on the next call. Later calls read it without the lock.
+template <typename T>
+class PerDevice {
+ public:
+  // `make(dev, &value)` returns cudaSuccess once it has stored the value.
+  template <typename F>
+  cudaError_t get(F&& make, T* out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (!ready_[dev].load(std::memory_order_acquire)) {
+      std::lock_guard<std::mutex> lock(mu_);
+      if (!ready_[dev].load(std::memory_order_relaxed)) {
+        e = make(dev, &val_[dev]);
+        if (e != cudaSuccess) return e;
+        ready_[dev].store(true, std::memory_order_release);
+      }
+    }
+    *out = val_[dev];
+    return cudaSuccess;
   }
-  return cached[dev];
+
+ private:
+  std::mutex mu_;
+  std::atomic<bool> ready_[kMaxDevices] = {};
+  T val_[kMaxDevices] = {};
+};
+
+// SM count of the current device (148 on B200; 148 if the query fails).
+inline int sm_count() {
+  static PerDevice<int> cache;
+  int n = 0;
+  const cudaError_t e = cache.get(
+      [](int dev, int* v) {
+        int c = 0;
+        const cudaError_t r = cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev);
+        if (r != cudaSuccess || c <= 0) return r != cudaSuccess ? r : cudaErrorInvalidValue;
+        *v = c;
+        return cudaSuccess;
+      },
+      &n);
+  return e == cudaSuccess ? n : 148;
 }
 
 }  // namespace lbq
+
+// LBQ_OK for cudaSuccess; otherwise records e as the calling thread's last CUDA error
+// (lbq_last_cuda_error) and returns LBQ_ERR_CUDA (api.cu).
+lbq_status lbq_cuda_status(cudaError_t e);
 
 // Launch helpers implemented in the individual .cu files; all return cudaError_t
 // from cudaGetLastError() after the launch.
@@ -112,6 +155,10 @@ cudaError_t lbq_launch_rht_signs(uint64_t seed, int64_t K, int8_t* D, cudaStream
 cudaError_t lbq_launch_hadamard(const uint16_t* x, const int8_t* D, int64_t M, int64_t K,
                                 float* out, cudaStream_t s);
 size_t lbq_gemv_workspace(const lbq_weights* w);
+// Every argument check lbq_gemv makes except the workspace's, with the same statuses
+// (api.cu).
+lbq_status lbq_validate_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D,
+                             const uint16_t* y);
 // Device address of the word bounded device waits report to (current device), or NULL.
 unsigned* lbq_fault_word();
 // Launches the kernel whose bounded wait runs out on purpose (selftest.cu).
@@ -119,6 +166,10 @@ cudaError_t lbq_launch_wait_selftest(cudaStream_t s);
 cudaError_t lbq_launch_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D,
                             uint16_t* y, void* ws, cudaStream_t s);
 size_t lbq_gemm_workspace(const lbq_weights* w, int64_t M);
+// The batched batch-1 products (gemv_batch.cu): workspace for a list of at most
+// LBQ_BATCH_MAX products, and one launch over such a list.
+size_t lbq_gemv_batch_ws(const lbq_product* ps, int32_t n);
+cudaError_t lbq_launch_gemv_batch(const lbq_product* ps, int32_t n, void* ws, cudaStream_t s);
 size_t lbq_gemm_tc_workspace(const lbq_weights* w, int64_t M);
 cudaError_t lbq_launch_gemm_tc(const lbq_weights* w, const uint16_t* X, int64_t M, uint16_t* Y,
                                void* ws, cudaStream_t s);

@@ -8,61 +8,49 @@
 // behind its back). This entry point needs no workspace argument: it uses
 // g_lbq_scratch below. The array costs LBQ_NOALLOC_SCRATCH_BYTES on every GPU that
 // loads the library, for the life of the process.
-#include <mutex>
-
 #include "lbq_common.cuh"
 
 namespace {
 
 static __device__ __align__(256) unsigned char g_lbq_scratch[LBQ_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
 // The array's device address, looked up once per device with that device current.
 // Host code must not pass the symbol itself to a kernel: on the host it is only a
 // stand-in, not a device address.
 lbq_status scratch_for_current_device(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LBQ_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_lbq_scratch) != cudaSuccess || !p) {
-      cudaGetLastError();
-      return LBQ_ERR_CUDA;
-    }
-    g_scratch_ptr[dev] = p;
+  static lbq::PerDevice<void*> addr;
+  const cudaError_t e = addr.get(
+      [](int, void** v) {
+        void* p = nullptr;
+        const cudaError_t r = cudaGetSymbolAddress(&p, g_lbq_scratch);
+        if (r != cudaSuccess) return r;
+        if (!p) return cudaErrorInvalidSymbol;
+        *v = p;
+        return cudaSuccess;
+      },
+      out);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return lbq_cuda_status(e);
   }
-  *out = g_scratch_ptr[dev];
   return LBQ_OK;
-}
-
-inline bool aligned(const void* p, uintptr_t a) {
-  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
 }
 
 }  // namespace
 
 extern "C" lbq_status lbq_gemv_noalloc(const lbq_weights* w, const uint16_t* x, const int8_t* D,
                                        uint16_t* y, void* stream) {
-  const size_t need = lbq_workspace_bytes(w, 1);  // 0 for an invalid descriptor
-  if (need > LBQ_NOALLOC_SCRATCH_BYTES) return LBQ_ERR_WORKSPACE;
-  if (need == 0) return lbq_gemv(w, x, D, y, nullptr, 0, stream);  // validates everything
-  // A scratch is needed, so the descriptor is valid; check the remaining arguments now,
-  // so that nothing is enqueued on a bad call.
-  if (!x || !y || (w->fmt == LBQ_Q2RHT && !D)) return LBQ_ERR_ARG;
-  if (!aligned(x, 16) || !aligned(y, 2) || (D && !aligned(D, 16))) return LBQ_ERR_ALIGN;
-  void* scratch = nullptr;
-  lbq_status st = scratch_for_current_device(&scratch);
+  // the same checks, in the same order, as lbq_gemv; then the scratch size
+  const lbq_status st = lbq_validate_gemv(w, x, D, y);
   if (st != LBQ_OK) return st;
-  // The array keeps whatever the previous call left; the product expects a zeroed
-  // workspace, so clear the part this call uses.
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(scratch, 0, need, s) != cudaSuccess) {
-    cudaGetLastError();
-    return LBQ_ERR_CUDA;
-  }
+  const size_t need = lbq_workspace_bytes(w, 1);
+  if (need > LBQ_NOALLOC_SCRATCH_BYTES) return LBQ_ERR_WORKSPACE;
+  if (need == 0) return lbq_gemv(w, x, D, y, nullptr, 0, stream);
+  void* scratch = nullptr;
+  const lbq_status sst = scratch_for_current_device(&scratch);
+  if (sst != LBQ_OK) return sst;
+  // Nothing needs clearing: the batch-1 product writes every slice sum before it reads
+  // it, and never touches the arrival counters at the array's start, which are zero
+  // since the library was loaded (static device memory starts zeroed).
   return lbq_gemv(w, x, D, y, scratch, LBQ_NOALLOC_SCRATCH_BYTES, stream);
 }

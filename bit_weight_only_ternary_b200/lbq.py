@@ -22,7 +22,9 @@ LBQ_OK, LBQ_ERR_ARG, LBQ_ERR_SHAPE, LBQ_ERR_ALIGN, LBQ_ERR_FORMAT, LBQ_ERR_CUDA,
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblbq.so")
 EXPORTS = ("lbq_status_string", "lbq_packed_layout", "lbq_pack", "lbq_unpack", "lbq_rht_signs",
            "lbq_hadamard", "lbq_workspace_bytes", "lbq_gemv", "lbq_gemm", "lbq_gemv_noalloc", "lbq_device_fault",
-           "lbq_selftest_wait")
+           "lbq_selftest_wait", "lbq_read_probe", "lbq_gemv_batch_workspace_bytes", "lbq_gemv_batch",
+           "lbq_last_cuda_error", "lbq_last_cuda_error_string")
+LBQ_BATCH_MAX = 256
 LBQ_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -32,10 +34,18 @@ class lbq_weights(ctypes.Structure):
                 ("code_stride", ctypes.c_int64), ("scale_stride", ctypes.c_int64)]
 
 
+class lbq_product(ctypes.Structure):
+    _fields_ = [("w", lbq_weights), ("x", ctypes.c_void_p), ("D", ctypes.c_void_p),
+                ("y", ctypes.c_void_p)]
+
+
 class LbqError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {lbq_status_string(status)} (status {status})")
+        extra = ""
+        if status == LBQ_ERR_CUDA:
+            extra = f": {_lib.lbq_last_cuda_error_string().decode()} ({_lib.lbq_last_cuda_error()})"
+        super().__init__(f"{where}: {lbq_status_string(status)} (status {status}){extra}")
 
 
 def _load():
@@ -58,6 +68,11 @@ def _load():
         "lbq_gemv_noalloc": (ctypes.c_int, [W, p, p, p, p]),
         "lbq_device_fault": (ctypes.c_int, [p]),
         "lbq_selftest_wait": (ctypes.c_int, [p]),
+        "lbq_read_probe": (ctypes.c_int, [p, sz, p, p]),
+        "lbq_gemv_batch_workspace_bytes": (sz, [ctypes.POINTER(lbq_product), i32]),
+        "lbq_gemv_batch": (ctypes.c_int, [ctypes.POINTER(lbq_product), i32, p, sz, p]),
+        "lbq_last_cuda_error": (i32, []),
+        "lbq_last_cuda_error_string": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -229,3 +244,51 @@ def lbq_gemv_noalloc(pw: PackedWeights, x: torch.Tensor, D=None, y=None,
     _check(_lib.lbq_gemv_noalloc(ctypes.byref(d), _ptr(x), _ptr(D), _ptr(y), _stream(stream)),
            "lbq_gemv_noalloc")
     return y
+
+
+def lbq_read_probe(buf: torch.Tensor, sink: torch.Tensor, nbytes: int | None = None,
+                   stream=None) -> None:
+    """Reads nbytes (default: all) of a device tensor once, XOR-folding the words into
+    sink (an int32 device tensor): the plain read-stream rate, a bandwidth denominator."""
+    n = buf.numel() * buf.element_size() if nbytes is None else int(nbytes)
+    _check(_lib.lbq_read_probe(_ptr(buf), n, _ptr(sink), _stream(stream)), "lbq_read_probe")
+
+
+class ProductList:
+    """A host array of lbq_product records for lbq_gemv_batch, built once from
+    (packed weights, x, D or None, y) tuples; the tensors must outlive its use."""
+
+    def __init__(self, items):
+        self.items = list(items)
+        self.arr = (lbq_product * len(self.items))()
+        for i, (pw, x, D, y) in enumerate(self.items):
+            self.arr[i].w = pw.desc()
+            self.arr[i].x = x.data_ptr()
+            self.arr[i].D = None if D is None else D.data_ptr()
+            self.arr[i].y = y.data_ptr()
+
+    def __len__(self):
+        return len(self.items)
+
+
+def lbq_gemv_batch_workspace_bytes(plist: ProductList) -> int:
+    return int(_lib.lbq_gemv_batch_workspace_bytes(plist.arr, len(plist)))
+
+
+def lbq_gemv_batch(plist: ProductList, workspace=None, stream=None) -> None:
+    """Every product of the list (independent batch-1 products, see include/lbq.h), one
+    persistent launch per LBQ_BATCH_MAX products. The workspace's first 64 KB must be
+    zero when it is first used (workspace_for_batch gives such a buffer)."""
+    if workspace is None:
+        workspace = workspace_for_batch(plist)
+    wsb = workspace.numel() * workspace.element_size()
+    _check(_lib.lbq_gemv_batch(plist.arr, len(plist), _ptr(workspace), wsb, _stream(stream)),
+           "lbq_gemv_batch")
+
+
+def workspace_for_batch(plist: ProductList, device=None) -> torch.Tensor:
+    n = lbq_gemv_batch_workspace_bytes(plist)
+    if n == 0:
+        _check(LBQ_ERR_ARG, "lbq_gemv_batch_workspace_bytes")
+    dev = device or plist.items[0][1].device
+    return torch.zeros(((n + 15) // 16) * 16, dtype=torch.uint8, device=dev)

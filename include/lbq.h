@@ -124,6 +124,12 @@ typedef struct lbq_weights {
 /* Human-readable name of a status. Never NULL. Host only. */
 const char* lbq_status_string(lbq_status st);
 
+/* The CUDA runtime error (a cudaError_t value) behind the last LBQ_ERR_CUDA that a
+ * call returned on the calling host thread, or 0 if none has; and its text (never
+ * NULL). Host only; no CUDA call is made. */
+int32_t lbq_last_cuda_error(void);
+const char* lbq_last_cuda_error_string(void);
+
 /* Packed sizes for a K x N matrix in format `fmt` (host only, no CUDA call).
  * Any output pointer may be NULL. code_stride/scale_stride are the minimal
  * strides; with N4 = N rounded up to a multiple of four (the storage order groups
@@ -157,7 +163,10 @@ lbq_status lbq_rht_signs(uint64_t seed, int64_t K, int8_t* D, void* stream);
 /* Block random Hadamard transform of M rows of bf16 activations ([rht]):
  * out[m][512c+i] = 2^-4.5 * sum_j (-1)^popcount(i&j) * D[512c+j] * x[m][512c+j].
  * x is [M][K] bf16 (row stride K), out is [M][K] fp32, K % 512 == 0.
- * Computed with a 9-stage butterfly in shared memory, in fp32. */
+ * One warp per (row, 512-block) computes the 9-stage butterfly in fp32: four stages
+ * within each lane's 16 values in registers, five across lanes with warp shuffles.
+ * (Output is fp32 only, and D is a device array only: the rotated activations feed
+ * fp32 arithmetic, and the signs are made on the device from the seed.) */
 lbq_status lbq_hadamard(const uint16_t* x, const int8_t* D, int64_t M, int64_t K,
                         float* out, void* stream);
 
@@ -187,12 +196,57 @@ lbq_status lbq_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D, ui
  * ([M][K], row stride K) into bf16 Y ([M][N], row stride N). Ternary weights:
  * up to 3 rows run as one batch-1 product per row (lbq_gemv's kernels, in stream
  * order), more rows dequantise weight tiles into tensor memory and run tcgen05
- * fp16 MMAs with fp32 accumulation (the activations are scaled into fp16 by an exact
- * power of two per row). 1-bit and 2-bit weights: a CUDA-core kernel that streams
- * the weights once for up to 8 rows at a time. Same formats, D and workspace rules
- * as lbq_gemv (workspace for this M, from lbq_workspace_bytes). */
+ * fp16 MMAs with fp32 accumulation. The activations are scaled into fp16 by an exact
+ * power of two per row; a row whose values do not all convert exactly (its values
+ * span more than about 2^31) is recomputed in fp32 on the CUDA cores, which is
+ * slower but keeps the same accuracy. 1-bit and 2-bit weights: a CUDA-core kernel
+ * in which each warp decodes a weight row's blocks once for up to 8 activation rows.
+ * Same formats, D and workspace rules as lbq_gemv (workspace for this M, from
+ * lbq_workspace_bytes). */
 lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const int8_t* D,
                     uint16_t* Y, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Measurement hook: reads `bytes` of device memory at p once (16-byte loads that do
+ * not allocate in L1, four CTAs per SM) and XORs the words read into *sink (device,
+ * 4-byte aligned), so that nothing is skipped. Its rate is the ceiling a plain read
+ * stream reaches on this GPU, the third denominator (after the nominal figure and
+ * the measured copy rate) for the products' weight streams. Not part of the method.
+ * Errors: LBQ_ERR_ARG (nulls), LBQ_ERR_SHAPE (bytes 0 or not a multiple of 16),
+ * LBQ_ERR_ALIGN (p not 16-byte aligned), LBQ_ERR_CUDA. */
+lbq_status lbq_read_probe(const void* p, size_t bytes, uint32_t* sink, void* stream);
+
+/* Most products one launch of lbq_gemv_batch takes (longer lists run as several). */
+#define LBQ_BATCH_MAX 256
+
+/* One batch-1 product of a list: y = W_hat x (W_hat from w; D for LBQ_Q2RHT, else NULL). */
+typedef struct lbq_product {
+  lbq_weights w;
+  const uint16_t* x;  /* device bf16 [K]                          */
+  const int8_t* D;    /* device int8 [K] rotation signs, or NULL   */
+  uint16_t* y;        /* device bf16 [N]                           */
+} lbq_product;
+
+/* Bytes of workspace lbq_gemv_batch needs for this list (0 on bad arguments). Its
+ * first 64 KB hold counters under the same rule as lbq_workspace_bytes: zero when the
+ * workspace is first used, zero again after every completed call. */
+size_t lbq_gemv_batch_workspace_bytes(const lbq_product* ps, int32_t n);
+
+/* n independent batch-1 products, each with the result lbq_gemv gives it, computed by
+ * one persistent launch per LBQ_BATCH_MAX products ([tern] §1.2, [block] §2.1-2.2,
+ * [sign], [rht]: the same lookup arithmetic as lbq_gemv). One CTA per SM stays
+ * resident for the whole list, so no product pays for a launch, a dependency wait or
+ * a separate split-K kernel, and the weight stream runs on between products: while
+ * the compute warps rebuild their lookup table for a product, a helper warp has the
+ * next product's weights fetched into L2 and adds up the previous product's slice
+ * sums. The products must be independent: no x or D of the list may overlap any y
+ * of the list, and no two y may overlap (checked on the host: LBQ_ERR_ARG). Products
+ * may use different formats and shapes. `ps` is host memory, read during the call
+ * only. The launch is cooperative (all CTAs resident at once). Workspace as
+ * lbq_gemv_batch_workspace_bytes; calls sharing one workspace must not overlap.
+ * Errors: those of lbq_gemv for any product, LBQ_ERR_ARG (ps NULL, n < 1, overlap),
+ * LBQ_ERR_WORKSPACE, LBQ_ERR_CUDA. */
+lbq_status lbq_gemv_batch(const lbq_product* ps, int32_t n, void* workspace,
+                          size_t workspace_bytes, void* stream);
 
 /* Size of the scratch array that lbq_gemv_noalloc uses (4 MiB). */
 #define LBQ_NOALLOC_SCRATCH_BYTES (4u << 20)
@@ -202,7 +256,8 @@ lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const in
  * kernels (on an mbarrier, for a TMA copy or a slot) is bounded by about 2 s; a
  * wait that runs out records a non-zero *code (3: shared-memory layout of the
  * batch-1 product, 4-9: tensor-core product stages, 10: the batch-1 product's
- * weight copies, 11: lbq_selftest_wait) and the kernel returns early with
+ * weight copies, 11: lbq_selftest_wait, 12: lbq_gemv_batch's waits on other CTAs,
+ * 13: lbq_gemv_batch's shared-memory layout) and the kernel returns early with
  * incomplete outputs instead of hanging. Synchronises the device.
  * Returns LBQ_OK with *code = 0 when no wait gave up, LBQ_ERR_DEVICE_WAIT with the
  * code otherwise. Errors: LBQ_ERR_ARG (code NULL), LBQ_ERR_CUDA. */
@@ -227,8 +282,10 @@ lbq_status lbq_selftest_wait(void* stream);
  * needs more scratch than that (lbq_workspace_bytes(w, 1)) returns
  * LBQ_ERR_WORKSPACE and enqueues nothing; use lbq_gemv with your own workspace
  * then. The call allocates nothing: no cudaMalloc, no cudaFree, no allocating
- * library routine. It clears the part of the array it uses (an asynchronous
- * memset on `stream`) before the product.
+ * library routine. It enqueues the product's kernels only: the product writes every
+ * scratch value before reading it, and the array's arrival counters, which it never
+ * writes, are zero from the moment the library is loaded, so there is nothing to
+ * clear between calls.
  *
  * The first call on each device looks up the array's device address (with that
  * device current) and caches it; make that first call before any stream capture.

@@ -66,7 +66,7 @@ def test_noalloc_rejects_products_needing_more_scratch(L):
     lib = L.lib()
     fake = ctypes.c_void_p(1 << 40)
     found = 0
-    for fmt, K, N in [(3, 1 << 21, 1), (1, 5120, 1 << 20), (2, 5120, 1 << 20), (1, 17408, 1 << 20)]:
+    for fmt, K, N in [(3, 1 << 21, 1), (1, 5120, 1 << 19), (2, 5120, 1 << 19), (1, 17408, 1 << 19)]:
         cs, ss, _, _ = L.lbq_packed_layout(fmt, K, 1)
         d = L.lbq_weights(fmt, 0, K, N, fake.value, None if fmt == 1 else fake.value, cs, ss)
         need = lib.lbq_workspace_bytes(ctypes.byref(d), 1)
@@ -75,7 +75,19 @@ def test_noalloc_rejects_products_needing_more_scratch(L):
             st = lib.lbq_gemv_noalloc(ctypes.byref(d), fake, fake, fake, None)
             assert st == L.LBQ_ERR_WORKSPACE
     assert found, "no test shape needs more than the fixed scratch"
-    # invalid arguments are refused with the same statuses as lbq_gemv
+    # invalid arguments are refused with the same statuses as lbq_gemv, checked before
+    # the scratch size: a null x or y, or a misaligned x, on a product too large for the
+    # array is an argument error, not a scratch error
+    cs, _, _, _ = L.lbq_packed_layout(1, 5120, 1)
+    big = L.lbq_weights(1, 0, 5120, 1 << 20, fake.value, None, cs, 0)
+    assert lib.lbq_gemv_noalloc(ctypes.byref(big), None, None, fake, None) == L.LBQ_ERR_ARG
+    assert lib.lbq_gemv_noalloc(ctypes.byref(big), fake, None, None, None) == L.LBQ_ERR_ARG
+    assert lib.lbq_gemv_noalloc(ctypes.byref(big), ctypes.c_void_p(fake.value + 2), None, fake,
+                                None) == L.LBQ_ERR_ALIGN
+    # more rows than a split product may have: a shape error, as from lbq_gemv
+    huge = L.lbq_weights(1, 0, 5120, (1 << 19) + 4, fake.value, None, cs, 0)
+    assert lib.lbq_gemv_noalloc(ctypes.byref(huge), fake, None, fake, None) == L.LBQ_ERR_SHAPE
+    assert lib.lbq_gemv(ctypes.byref(huge), fake, None, fake, fake, 1 << 30, None) == L.LBQ_ERR_SHAPE
     d = L.lbq_weights(1, 0, 500, 4, fake.value, None, 32, 0)
     assert lib.lbq_gemv_noalloc(ctypes.byref(d), fake, None, fake, None) == L.LBQ_ERR_SHAPE
     assert lib.lbq_gemv_noalloc(None, fake, None, fake, None) == L.LBQ_ERR_ARG
