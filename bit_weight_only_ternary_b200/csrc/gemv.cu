@@ -90,6 +90,7 @@ struct Args {
   const uint16_t* x;
   const int8_t* D;
   uint16_t* y;
+  float* y32;       // if set, y is written here as fp32 (no bf16 rounding) instead
   float* part;      // [KS][N] slice sums (KS > 1)
   int KS;           // number of slices
   int G;            // CTAs per slice
@@ -98,11 +99,13 @@ struct Args {
 };
 
 // One CTA: kWarps consumer warps and one warp that issues the weight copies. At most
-// 112 registers a thread (544 x 112 = 60928 of the SM's 65536), so that a CTA of the
-// split-K sum kernel (128 threads x 32) always fits beside it. tm_c / tm_s: the
-// codes / scales as tensor maps with a box of kSub units (tm_c1 / tm_s1: one unit).
+// 96 registers a thread: the register file is split between the SM's four schedulers,
+// and the CTA's 17 warps put five on one of them (5 x 32 x 96 = 15360 of its 16384,
+// which also leaves room for a warp of the split-K sum kernel at 32 registers).
+// tm_c / tm_s: the codes / scales as tensor maps with a box of kSub units (tm_c1 /
+// tm_s1: one unit).
 template <int FMT>
-__global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtensorMap tm_c,
+__global__ void __maxnreg__(96) gemv_lut_kernel(const __grid_constant__ CUtensorMap tm_c,
                                                  const __grid_constant__ CUtensorMap tm_s,
                                                  const __grid_constant__ CUtensorMap tm_c1,
                                                  const __grid_constant__ CUtensorMap tm_s1,
@@ -247,57 +250,28 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
   const int wl = lane_word<FMT>(lane, nb);
   const int wq = lane_word<FMT>(lane & ~7, nb);
   const uint32_t woff = 16u * static_cast<uint32_t>(wl >= 0 ? wl : (wq >= 0 ? wq : 0));
-  const int sblk = wl < 0 ? 0 : (FMT == LBQ_SIGN1 ? (lane >> 2) : (lane >> 1));
-  const uint32_t soff = kScaleOff + 8u * static_cast<uint32_t>(sblk);
   const uint32_t lanereg = tbase | static_cast<uint32_t>(lane * 4);
-  const int src6 = (lane & ~7) | 6;  // ternary: the lane holding this block's scale word
+  // The block scales this lane multiplies after the in-block butterfly stages
+  // (unit_sum): ternary, the scale words of rows R, R + 1 of its block (word 6 of the
+  // block, inside the codes); 1-bit, group G's four scales of its block; 2-bit, groups
+  // G and G + 1's. Offsets within a unit's codes / scales in the ring slot.
+  uint32_t s_off;
+  if (FMT == LBQ_TERN5) {
+    const int R = 8 * (lane & 1) + 4 * ((lane >> 1) & 1) + 2 * ((lane >> 2) & 1);
+    const int b = (lane >> 3) < nb ? (lane >> 3) : nb - 1;
+    s_off = static_cast<uint32_t>((R >> 2) * T::kGroupBytes + 16 * (7 * b + 6) + 4 * (R & 3));
+  } else {
+    const int b = FMT == LBQ_SIGN1 ? (lane >> 2) : (lane >> 1);
+    const int bb = b < nb ? b : nb - 1;
+    const int G = FMT == LBQ_SIGN1 ? 2 * (lane & 1) + ((lane >> 1) & 1) : 2 * (lane & 1);
+    s_off = kScaleOff + static_cast<uint32_t>(G * T::kScaleBytes + 8 * bb);
+  }
+  // the row unit_sum leaves in this lane (lanes < 16 store it)
+  const int rloc = 8 * (lane & 1) + 4 * ((lane >> 1) & 1) + 2 * ((lane >> 2) & 1) + ((lane >> 3) & 1);
   const int64_t NR = a.N;
   float* const part_j = a.part + static_cast<int64_t>(j) * NR;
   uint16_t* const y = a.y;
   const bool direct = a.KS == 1;
-  // one unit: table lookups, block scales, transpose-reduce, store
-  auto unit = [&](const uint4 (&b)[4], const uint2 (&sb)[4], int32_t t) {
-    float acc[kRows];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint4 v = b[q];
-      float2 p01 = lookup_pair(v.x, v.y, lanereg);
-      float2 p23 = lookup_pair(v.z, v.w, lanereg);
-      uint32_t s01, s23;
-      if (kSepScales) {
-        s01 = sb[q].x;
-        s23 = sb[q].y;
-      } else {
-        s01 = __shfl_sync(0xffffffffu, __byte_perm(v.x, v.y, 0x7632), src6);
-        s23 = __shfl_sync(0xffffffffu, __byte_perm(v.z, v.w, 0x7632), src6);
-      }
-      p01 = __fmul2_rn(p01, h2_to_f2(s01));
-      p23 = __fmul2_rn(p23, h2_to_f2(s23));
-      acc[4 * q] = p01.x;
-      acc[4 * q + 1] = p01.y;
-      acc[4 * q + 2] = p23.x;
-      acc[4 * q + 3] = p23.y;
-    }
-    // transpose-reduce: afterwards acc[0] is row (lane & 15), summed over all lanes
-#pragma unroll
-    for (int d = kRows / 2; d >= 1; d >>= 1) {
-      const bool up = (lane & d) != 0;
-#pragma unroll
-      for (int r = 0; r < d; ++r) {
-        const float send = up ? acc[r] : acc[r + d];
-        const float keep = up ? acc[r + d] : acc[r];
-        acc[r] = keep + __shfl_xor_sync(0xffffffffu, send, d);
-      }
-    }
-    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 16);
-    const int64_t row = static_cast<int64_t>(u_lo + warp + kWarps * t) * kRows + lane;
-    if (lane < kRows && row < NR) {
-      if (direct)
-        y[row] = f32_to_bf16_bits(acc[0]);
-      else
-        part_j[row] = acc[0];
-    }
-  };
   // ---- consumers: warp w takes units w, w + kWarps, ...; unit tg sits in slot
   // sequence number tg / kSub at place tg % kSub (= w % kSub)
   const uint32_t sub = static_cast<uint32_t>(warp % kSub);
@@ -307,20 +281,31 @@ __global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ CUtenso
   for (int32_t t = 0; t < nt; ++t) {
     if (!mbar_wait(full0 + 8 * slot, round & 1, a.fault, kFaultRing)) break;
     const uint32_t src = slot_addr(slot);
-    uint4 b[4];
-    uint2 sb[4];
+    UnitRegs r;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      b[q] = lds_v4(src + (4 * sub + q) * T::kGroupBytes + woff);
-      sb[q] = kSepScales ? lds_v2(src + soff + (4 * sub + q) * T::kScaleBytes) : make_uint2(0u, 0u);
+    for (int q = 0; q < 4; ++q) r.w[q] = lds_v4(src + (4 * sub + q) * T::kGroupBytes + woff);
+    if (FMT == LBQ_TERN5) {
+      r.s[0] = lds_v2(src + 4 * sub * T::kGroupBytes + s_off);
+    } else {
+      r.s[0] = lds_v2(src + 4 * sub * T::kScaleBytes + s_off);
+      if (FMT == LBQ_Q2RHT) r.s[1] = lds_v2(src + (4 * sub + 1) * T::kScaleBytes + s_off);
     }
-    unit(b, sb, t);
-    // The warp has used its words: the slot goes back to the copies (the warp barrier
-    // and the proxy fence order these reads before the copy engine's next writes).
+    // The warp has its words: the slot goes back to the copies (the warp barrier and
+    // the proxy fence order these reads before the copy engine's next writes).
     __syncwarp();
     if (lane == 0) {
       fence_proxy_async_smem();
       mbar_arrive(empty0 + 8 * slot);
+    }
+    const float v = unit_sum<FMT>(r, lanereg, lane);
+    const int64_t row = static_cast<int64_t>(u_lo + warp + kWarps * t) * kRows + rloc;
+    if (lane < kRows && row < NR) {
+      if (!direct)
+        part_j[row] = v;
+      else if (a.y32)
+        a.y32[row] = v;
+      else
+        y[row] = f32_to_bf16_bits(v);
     }
     slot += kGroups;
     if (slot >= S) {
@@ -344,7 +329,7 @@ constexpr int kSumThreads = 128, kSumRun = 8;
 template <bool kPairs>
 __global__ void __maxnreg__(32)
     splitk_sum_kernel(const float* __restrict__ part, int KS, int64_t N, int logP,
-                      uint16_t* __restrict__ y) {
+                      uint16_t* __restrict__ y, float* __restrict__ y32) {
   pdl_launch_dependents();
   pdl_wait();
   using V = typename std::conditional<kPairs, float2, float>::type;
@@ -388,7 +373,14 @@ __global__ void __maxnreg__(32)
       if (kPairs) ay += __shfl_down_sync(0xffffffffu, ay, o, P);
     }
     if (idx < total && sg == 0) {
-      if (kPairs) {
+      if (y32) {
+        if (kPairs) {
+          y32[2 * e] = ax;
+          y32[2 * e + 1] = ay;
+        } else {
+          y32[e] = ax;
+        }
+      } else if (kPairs) {
         y[2 * e] = f32_to_bf16_bits(ax);
         y[2 * e + 1] = f32_to_bf16_bits(ay);
       } else {
@@ -407,7 +399,7 @@ int slices_of(const lbq_weights* w) {
 }
 
 template <int FMT>
-cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uint16_t* y, void* ws,
+cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uint16_t* y, float* y32, void* ws,
                    cudaStream_t s) {
   static PerDevice<bool> configured;  // the kernel's shared-memory limit, set once per device
   bool ok = false;
@@ -425,6 +417,7 @@ cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uin
   a.x = x;
   a.D = D;
   a.y = y;
+  a.y32 = y32;
   a.KS = slices_of(w);
   a.nblk = static_cast<int>(w->K / (FMT == LBQ_Q2RHT ? kQ2Block : kTernBlock));
   a.fault = lbq_fault_word();
@@ -498,8 +491,8 @@ cudaError_t launch(const lbq_weights* w, const uint16_t* x, const int8_t* D, uin
   cfg2.dynamicSmemBytes = 0;
   const float* part = a.part;
   const int64_t N = w->N;
-  return pairs ? cudaLaunchKernelEx(&cfg2, splitk_sum_kernel<true>, part, a.KS, N, logP, y)
-               : cudaLaunchKernelEx(&cfg2, splitk_sum_kernel<false>, part, a.KS, N, logP, y);
+  return pairs ? cudaLaunchKernelEx(&cfg2, splitk_sum_kernel<true>, part, a.KS, N, logP, y, y32)
+               : cudaLaunchKernelEx(&cfg2, splitk_sum_kernel<false>, part, a.KS, N, logP, y, y32);
 }
 
 }  // namespace
@@ -530,10 +523,10 @@ size_t lbq_gemv_workspace(const lbq_weights* w) {
 }
 
 cudaError_t lbq_launch_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D,
-                            uint16_t* y, void* ws, cudaStream_t s) {
+                            uint16_t* y, float* y32, void* ws, cudaStream_t s) {
   switch (w->fmt) {
-    case LBQ_TERN5: return launch<LBQ_TERN5>(w, x, D, y, ws, s);
-    case LBQ_SIGN1: return launch<LBQ_SIGN1>(w, x, D, y, ws, s);
-    default: return launch<LBQ_Q2RHT>(w, x, D, y, ws, s);
+    case LBQ_TERN5: return launch<LBQ_TERN5>(w, x, D, y, y32, ws, s);
+    case LBQ_SIGN1: return launch<LBQ_SIGN1>(w, x, D, y, y32, ws, s);
+    default: return launch<LBQ_Q2RHT>(w, x, D, y, y32, ws, s);
   }
 }

@@ -61,8 +61,9 @@ __device__ __forceinline__ int digit_weight(int slot, int l, int e, int nb) {
   const int w = lane_word<FMT>(l, nb);
   if (w < 0) return -1;
   if (FMT == LBQ_TERN5) {
-    const int bb = w / 7, c = 4 * (w % 7) + slot;  // byte within the 28-byte block
-    if (c >= kTernCodeBytes) return -1;            // the block's fp16 scale
+    // lane l holds word l % 8 of block l / 8 (lane_word), so no division is needed
+    const int bb = l >> 3, c = 4 * (l & 7) + slot;  // byte within the 28-byte block
+    if (c >= kTernCodeBytes) return -1;              // the block's fp16 scale
     const int kb = 5 * c + e;
     return kb < kTernBlock ? bb * kTernBlock + kb : -1;
   } else if (FMT == LBQ_SIGN1) {
@@ -258,6 +259,64 @@ __device__ __forceinline__ void build_table(int nb, uint32_t tbase, const float*
       }
     }
   }
+}
+
+// One 16-row unit (four groups of four rows) of one slice, as one lane holds it: its
+// word of each group's four rows and the block scales it multiplies after the in-block
+// stages of the butterfly (see unit_sum).
+struct UnitRegs {
+  uint4 w[4];   // the lane's word of each group's four rows
+  uint2 s[2];   // scales: ternary s[0] = scale words of rows R, R+1; 1-bit s[0] = group
+                // G's four scales of the lane's block; 2-bit s[0], s[1] = groups G, G + 1
+};
+
+// One transpose-reduce stage: c values -> c / 2; the lane keeps the upper half of the
+// row range if its bit d is set, the lower half otherwise, and adds its partner's.
+template <int C>
+__device__ __forceinline__ void tr_stage(float (&acc)[16], int lane, int d) {
+  const bool up = (lane & d) != 0;
+#pragma unroll
+  for (int r = 0; r < C / 2; ++r) {
+    const float send = up ? acc[r] : acc[r + C / 2];
+    const float keep = up ? acc[r + C / 2] : acc[r];
+    acc[r] = keep + __shfl_xor_sync(0xffffffffu, send, d);
+  }
+}
+
+// Lookups, block scales and the reduction of one unit; returns the sum of row
+// 8 b0 + 4 b1 + 2 b2 + b3 of the unit in every lane (b_k = bit k of the lane).
+template <int FMT>
+__device__ __forceinline__ float unit_sum(const UnitRegs& r, uint32_t lanereg, int lane) {
+  float acc[16];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 p01 = lookup_pair(r.w[q].x, r.w[q].y, lanereg);
+    const float2 p23 = lookup_pair(r.w[q].z, r.w[q].w, lanereg);
+    acc[4 * q] = p01.x;
+    acc[4 * q + 1] = p01.y;
+    acc[4 * q + 2] = p23.x;
+    acc[4 * q + 3] = p23.y;
+  }
+  tr_stage<16>(acc, lane, 1);
+  if (FMT == LBQ_Q2RHT) {  // 2 lanes a block: rows R .. R + 7 (two groups)
+    const float2 s0 = h2_to_f2(r.s[0].x), s1 = h2_to_f2(r.s[0].y);
+    const float2 s2 = h2_to_f2(r.s[1].x), s3 = h2_to_f2(r.s[1].y);
+    acc[0] *= s0.x; acc[1] *= s0.y; acc[2] *= s1.x; acc[3] *= s1.y;
+    acc[4] *= s2.x; acc[5] *= s2.y; acc[6] *= s3.x; acc[7] *= s3.y;
+  }
+  tr_stage<8>(acc, lane, 2);
+  if (FMT == LBQ_SIGN1) {  // 4 lanes a block: rows R .. R + 3 (one group)
+    const float2 s0 = h2_to_f2(r.s[0].x), s1 = h2_to_f2(r.s[0].y);
+    acc[0] *= s0.x; acc[1] *= s0.y; acc[2] *= s1.x; acc[3] *= s1.y;
+  }
+  tr_stage<4>(acc, lane, 4);
+  if (FMT == LBQ_TERN5) {  // 8 lanes a block (7 with words): rows R, R + 1
+    const float2 s = h2_to_f2(__byte_perm(r.s[0].x, r.s[0].y, 0x7632));
+    acc[0] *= s.x;
+    acc[1] *= s.y;
+  }
+  tr_stage<2>(acc, lane, 8);
+  return acc[0] + __shfl_xor_sync(0xffffffffu, acc[0], 16);
 }
 
 }  // namespace lut
