@@ -236,7 +236,16 @@ lbq_status lbq_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D, ui
   Layout L;
   lbq_status st = check_product(w, x, 1, D, y, workspace, workspace_bytes, &L);
   if (st != LBQ_OK) return st;
-  return from_cuda(lbq_launch_gemv(w, x, D, y, workspace, as_stream(stream)));
+  return from_cuda(lbq_launch_gemv(w, x, D, y, nullptr, workspace, as_stream(stream)));
+}
+
+lbq_status lbq_gemv_f32(const lbq_weights* w, const uint16_t* x, const int8_t* D, float* y,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  Layout L;
+  lbq_status st = check_product(w, x, 1, D, y, workspace, workspace_bytes, &L);
+  if (st != LBQ_OK) return st;
+  if (!aligned(y, 4)) return LBQ_ERR_ALIGN;
+  return from_cuda(lbq_launch_gemv(w, x, D, nullptr, y, workspace, as_stream(stream)));
 }
 
 size_t lbq_gemv_batch_workspace_bytes(const lbq_product* ps, int32_t n) {
@@ -277,7 +286,7 @@ lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const in
     // one batch-1 product per token, in stream order (they share the workspace)
     for (int64_t m = 0; m < M; ++m) {
       const cudaError_t e =
-          lbq_launch_gemv(w, X + m * w->K, D, Y + m * w->N, workspace, as_stream(stream));
+          lbq_launch_gemv(w, X + m * w->K, D, Y + m * w->N, nullptr, workspace, as_stream(stream));
       if (e != cudaSuccess) return lbq_cuda_status(e);
     }
     return LBQ_OK;

@@ -163,8 +163,9 @@ lbq_status lbq_validate_gemv(const lbq_weights* w, const uint16_t* x, const int8
 unsigned* lbq_fault_word();
 // Launches the kernel whose bounded wait runs out on purpose (selftest.cu).
 cudaError_t lbq_launch_wait_selftest(cudaStream_t s);
+// y (bf16) or, when y32 is set, y32 (fp32, no rounding) receives the product.
 cudaError_t lbq_launch_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D,
-                            uint16_t* y, void* ws, cudaStream_t s);
+                            uint16_t* y, float* y32, void* ws, cudaStream_t s);
 size_t lbq_gemm_workspace(const lbq_weights* w, int64_t M);
 // The batched batch-1 products (gemv_batch.cu): workspace for a list of at most
 // LBQ_BATCH_MAX products, and one launch over such a list.

@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblbq.so")
 EXPORTS = ("lbq_status_string", "lbq_packed_layout", "lbq_pack", "lbq_unpack", "lbq_rht_signs",
            "lbq_hadamard", "lbq_workspace_bytes", "lbq_gemv", "lbq_gemm", "lbq_gemv_noalloc", "lbq_device_fault",
            "lbq_selftest_wait", "lbq_read_probe", "lbq_gemv_batch_workspace_bytes", "lbq_gemv_batch",
-           "lbq_last_cuda_error", "lbq_last_cuda_error_string")
+           "lbq_last_cuda_error", "lbq_last_cuda_error_string", "lbq_gemv_f32")
 LBQ_BATCH_MAX = 256
 LBQ_NOALLOC_SCRATCH_BYTES = 4 << 20
 
@@ -64,6 +64,7 @@ def _load():
         "lbq_hadamard": (ctypes.c_int, [p, p, i64, i64, p, p]),
         "lbq_workspace_bytes": (sz, [W, i64]),
         "lbq_gemv": (ctypes.c_int, [W, p, p, p, p, sz, p]),
+        "lbq_gemv_f32": (ctypes.c_int, [W, p, p, p, p, sz, p]),
         "lbq_gemm": (ctypes.c_int, [W, p, i64, p, p, p, sz, p]),
         "lbq_gemv_noalloc": (ctypes.c_int, [W, p, p, p, p]),
         "lbq_device_fault": (ctypes.c_int, [p]),
@@ -215,6 +216,20 @@ def lbq_gemv(pw: PackedWeights, x: torch.Tensor, D=None, y=None, workspace=None,
     wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_lib.lbq_gemv(ctypes.byref(d), _ptr(x), _ptr(D), _ptr(y), _ptr(workspace), wsb,
                          _stream(stream)), "lbq_gemv")
+    return y
+
+
+def lbq_gemv_f32(pw: PackedWeights, x: torch.Tensor, D=None, y=None, workspace=None,
+                 stream=None) -> torch.Tensor:
+    """fp32 y [N] = W_hat x for bf16 x [K] (device), without the final bf16 rounding."""
+    if y is None:
+        y = torch.empty(pw.N, dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = workspace_for(pw, 1, x.device)
+    d = pw.desc()
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.lbq_gemv_f32(ctypes.byref(d), _ptr(x), _ptr(D), _ptr(y), _ptr(workspace), wsb,
+                             _stream(stream)), "lbq_gemv_f32")
     return y
 
 

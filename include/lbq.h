@@ -192,6 +192,13 @@ size_t lbq_workspace_bytes(const lbq_weights* w, int64_t M);
 lbq_status lbq_gemv(const lbq_weights* w, const uint16_t* x, const int8_t* D, uint16_t* y,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* lbq_gemv with an fp32 y [N] (4-byte aligned) in place of bf16: the same product,
+ * without the final rounding, for partial products that are added up afterwards
+ * (a layer whose input features are split over GPUs sums each GPU's partial y; a
+ * residual add). Same arguments, workspace and errors as lbq_gemv. */
+lbq_status lbq_gemv_f32(const lbq_weights* w, const uint16_t* x, const int8_t* D, float* y,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
 /* Batched product Y[m][n] = sum_k W_hat[n][k] X[m][k] for M rows of bf16 X
  * ([M][K], row stride K) into bf16 Y ([M][N], row stride N). Ternary weights:
  * up to 3 rows run as one batch-1 product per row (lbq_gemv's kernels, in stream
