@@ -55,7 +55,7 @@ WORKLOADS = {
 # the workloads measured beside the headline in a one-GPU run (plus the tiny GEMV)
 CONFIG_ORDER = ("tern_chained", "sign", "q2", "mixed", "mixed_chained", "gemm8", "gemm32",
                 "gemm512", "gemm4096")
-MODE_TEXT = {"batch": "independent products, one lbq_gemv_batch launch per pass",
+MODE_TEXT = {"batch": "independent products, one lbq_gemv_batch call per pass (one persistent launch per format)",
              "chained": "one lbq_gemv per product, each chained to the previous",
              "gemm": "one lbq_gemm per product"}
 FMT_NAME = {1: "ternary 5 trits/byte + fp16 scale per 128", 2: "1-bit sign + fp16 scale per 128",
@@ -337,10 +337,14 @@ class Pass:
 
 
 def launches_per_step(L, prods, mode):
-    """Our kernels per pass: one persistent launch per 256 products (batch), or per
-    product the GEMV plus the split-K sum when K spans several slices (chained)."""
+    """Our kernels per pass: one persistent launch per format and 256 products of it
+    (batch; the small install kernel that copies each launch's list is not counted), or
+    per product the GEMV plus the split-K sum when K spans several slices (chained)."""
     if mode == "batch":
-        return (len(prods) + L.LBQ_BATCH_MAX - 1) // L.LBQ_BATCH_MAX
+        per_fmt = {}
+        for p in prods:
+            per_fmt[p["fmt"]] = per_fmt.get(p["fmt"], 0) + 1
+        return sum((c + L.LBQ_BATCH_MAX - 1) // L.LBQ_BATCH_MAX for c in per_fmt.values())
     if mode == "chained":
         return sum(1 + (p["K"] > (1024 if p["fmt"] == L.LBQ_SIGN1 else 512)) for p in prods)
     return None  # lbq_gemm: 2 or 3 kernels per product, as the tile planner decides

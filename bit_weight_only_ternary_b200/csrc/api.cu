@@ -1,5 +1,7 @@
 // api.cu -- the C ABI (include/lbq.h): host-side validation, then one or more launches.
 // Nothing is enqueued unless every argument passes; launch failures map to LBQ_ERR_CUDA.
+#include <vector>
+
 #include "lbq_common.cuh"
 
 namespace {
@@ -265,12 +267,30 @@ lbq_status lbq_gemv_batch(const lbq_product* ps, int32_t n, void* workspace,
   const size_t need = lbq_gemv_batch_workspace_bytes(ps, n);
   if (!workspace || workspace_bytes < need) return LBQ_ERR_WORKSPACE;
   if (!aligned(workspace, 16)) return LBQ_ERR_ALIGN;
-  for (int32_t i = 0; i < n; i += LBQ_BATCH_MAX) {
-    const cudaError_t e = lbq_launch_gemv_batch(ps + i, n - i < LBQ_BATCH_MAX ? n - i : LBQ_BATCH_MAX,
-                                                workspace, as_stream(stream));
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      return lbq_cuda_status(e);
+  // The kernel runs one format a launch: a list of several runs as one launch (or
+  // chunk of LBQ_BATCH_MAX) per format present, in the list's order within each format.
+  bool one_format = true;
+  for (int32_t i = 1; i < n; ++i) one_format = one_format && ps[i].w.fmt == ps[0].w.fmt;
+  std::vector<lbq_product> sub;
+  for (const int32_t fmt : {LBQ_TERN5, LBQ_SIGN1, LBQ_Q2RHT}) {
+    const lbq_product* list = ps;
+    int32_t count = n;
+    if (!one_format) {
+      sub.clear();
+      for (int32_t i = 0; i < n; ++i)
+        if (ps[i].w.fmt == fmt) sub.push_back(ps[i]);
+      list = sub.data();
+      count = static_cast<int32_t>(sub.size());
+    } else if (ps[0].w.fmt != fmt) {
+      continue;
+    }
+    for (int32_t i = 0; i < count; i += LBQ_BATCH_MAX) {
+      const cudaError_t e = lbq_launch_gemv_batch(
+          list + i, count - i < LBQ_BATCH_MAX ? count - i : LBQ_BATCH_MAX, workspace, as_stream(stream));
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        return lbq_cuda_status(e);
+      }
     }
   }
   return LBQ_OK;

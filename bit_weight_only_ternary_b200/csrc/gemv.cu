@@ -67,7 +67,7 @@ constexpr int kSub = 4;                       // units per ring slot (one tensor
 // (the dynamic window starts 1 KB into shared memory on sm_100) the x slice, the
 // mbarriers and the first ring slots, above it the other ring slots. A window that
 // starts at 0 puts everything above the table.
-constexpr uint32_t kXBytes = 4096;  // the slice of x as fp32 (up to 1024)
+constexpr uint32_t kXBytes = lut::kXsBytes;  // the padded slice of x as fp32
 constexpr int kMaxSlots = 32;
 // x and the mbarriers, rounded up so that the ring slots after them stay 128-byte
 // aligned, as tensor copies into shared memory require

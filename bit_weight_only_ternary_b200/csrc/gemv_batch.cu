@@ -60,7 +60,7 @@ constexpr int kPrefetchUnits = 4;
 #ifndef LBQ_BATCH_HELPER_PREFETCH
 #define LBQ_BATCH_HELPER_PREFETCH 0
 #endif
-constexpr uint32_t kXBytes = 4096;           // one x slice as fp32 (up to 1024)
+constexpr uint32_t kXBytes = lut::kXsBytes;  // one padded x slice as fp32
 constexpr int kXBufs = 3;                    // x slices in shared memory (the helper works 2 ahead)
 constexpr uint32_t kMiscBytes = kXBufs * kXBytes + 1024;  // x slices, flags
 constexpr uint32_t kDescSmem = 16384;        // the product list, copied to shared memory
@@ -371,15 +371,7 @@ __device__ __forceinline__ void x_slice_warp(const BProd& P, int32_t j, int nb, 
       v[i] = 8 * c < nb * kTernBlock ? __ldg(x8 + c) : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int i = 0; i < kChunks / 32; ++i) {
-      const int c = lane + 32 * i;
-      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-      float4* d = reinterpret_cast<float4*>(xs + 8 * c);
-      d[0] = make_float4(__uint_as_float(w[0] << 16), __uint_as_float(w[0] & 0xffff0000u),
-                         __uint_as_float(w[1] << 16), __uint_as_float(w[1] & 0xffff0000u));
-      d[1] = make_float4(__uint_as_float(w[2] << 16), __uint_as_float(w[2] & 0xffff0000u),
-                         __uint_as_float(w[3] << 16), __uint_as_float(w[3] & 0xffff0000u));
-    }
+    for (int i = 0; i < kChunks / 32; ++i) x_store8<FMT>(v[i], xs, lane + 32 * i);
   }
 }
 
@@ -558,6 +550,11 @@ __device__ __forceinline__ void xload_product(const BArgs& a, int p, float* xs, 
 
 // Format masks: the kernel is compiled once per set of formats a list holds, so that a
 // list of one format gets code (and registers) for that format alone.
+// The kernel is compiled once per format (kFmts = that format's bit): one kernel that
+// chose the format per product needed more registers than a thread has, and ran every
+// phase of a pass about twice as slowly (measured on a ternary list, as a function
+// call per product and inlined alike), so a list of several formats is run as one
+// launch per format (the products are independent).
 __host__ __device__ constexpr int fmt_bit(int fmt) { return 1 << (fmt - 1); }
 
 template <int kFmts>
@@ -660,10 +657,9 @@ __global__ void __maxnreg__(kMaxRegs) gemv_batch_kernel(const __grid_constant__ 
     bool ok = true;
     for (int p = 0; p < a.n; ++p) {
       if (tid == 0) st_release_cta(&fl->started, p + 1);
-      const int f = a.p[p].fmt;
-      if ((kFmts & fmt_bit(LBQ_TERN5)) && f == LBQ_TERN5) compute_product<LBQ_TERN5>(a, p, tbase, xbuf, fl, prep, tid, ok);
-      if ((kFmts & fmt_bit(LBQ_SIGN1)) && f == LBQ_SIGN1) compute_product<LBQ_SIGN1>(a, p, tbase, xbuf, fl, prep, tid, ok);
-      if ((kFmts & fmt_bit(LBQ_Q2RHT)) && f == LBQ_Q2RHT) compute_product<LBQ_Q2RHT>(a, p, tbase, xbuf, fl, prep, tid, ok);
+      compute_product<kFmts == fmt_bit(LBQ_TERN5)   ? LBQ_TERN5
+                      : kFmts == fmt_bit(LBQ_SIGN1) ? LBQ_SIGN1
+                                                    : LBQ_Q2RHT>(a, p, tbase, xbuf, fl, prep, tid, ok);
     }
     reduce_tail(a, fl, tid, ok);
   } else {
@@ -786,7 +782,7 @@ cudaError_t lbq_launch_gemv_batch(const lbq_product* ps, int32_t n, void* ws, cu
   cudaError_t e = mask == fmt_bit(LBQ_TERN5)   ? batch_grid<1>(&grid)
                   : mask == fmt_bit(LBQ_SIGN1) ? batch_grid<2>(&grid)
                   : mask == fmt_bit(LBQ_Q2RHT) ? batch_grid<4>(&grid)
-                                               : batch_grid<7>(&grid);
+                                               : cudaErrorInvalidValue;  // one format a launch
   if (e != cudaSuccess) return e;
   unsigned* fault = lbq_fault_word();
   if (!fault) return cudaErrorInvalidDevicePointer;
@@ -830,6 +826,5 @@ cudaError_t lbq_launch_gemv_batch(const lbq_product* ps, int32_t n, void* ws, cu
   }
   return mask == fmt_bit(LBQ_TERN5)   ? launch_batch<1>(a, grid, s)
          : mask == fmt_bit(LBQ_SIGN1) ? launch_batch<2>(a, grid, s)
-         : mask == fmt_bit(LBQ_Q2RHT) ? launch_batch<4>(a, grid, s)
-                                      : launch_batch<7>(a, grid, s);
+                                      : launch_batch<4>(a, grid, s);
 }

@@ -115,6 +115,28 @@ __device__ __forceinline__ float2 lookup_pair(uint32_t w0, uint32_t w1, uint32_t
   return __fadd2_rn(__fadd2_rn(e0, e1), __fadd2_rn(e2, e3));
 }
 
+// Position of weight k of a slice in the shared-memory x buffer: one pad float after
+// every 32 (1-bit, 2-bit) or two after every 128 (ternary). The table builders read x
+// 32 (1-bit), 16 (2-bit) or about 128 (ternary) weights apart across a warp's lanes;
+// unpadded, those reads fall on one bank (16-way conflicts for the 1-bit and 2-bit
+// formats, 4-way for ternary), padded on 16 or 32 different banks.
+template <int FMT>
+__device__ __forceinline__ int xs_pos(int k) {
+  return FMT == LBQ_TERN5 ? k + 2 * (k >> 7) : k + (k >> 5);
+}
+constexpr uint32_t kXsBytes = 4 * (1024 + 32);  // the largest padded slice (1-bit)
+
+// Eight bf16 activations (weights 8c .. 8c + 7 of the slice) stored as fp32.
+template <int FMT>
+__device__ __forceinline__ void x_store8(uint4 v, float* xs, int c) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    xs[xs_pos<FMT>(8 * c + 2 * q)] = __uint_as_float(w[q] << 16);
+    xs[xs_pos<FMT>(8 * c + 2 * q + 1)] = __uint_as_float(w[q] & 0xffff0000u);
+  }
+}
+
 // The x slice of slice j, loaded by x_issue with plain loads and stored to shared memory
 // as fp32 by x_store (the 2-bit format: rotated by one warp on the way).
 struct XLoad {
@@ -158,23 +180,11 @@ __device__ __forceinline__ void x_store(const XLoad& r, float* xs, int tid) {
         v[i] = sgn < 0 ? -xv : xv;
       }
       fwht512_warp(v);
-      float4* d = reinterpret_cast<float4*>(xs + 16 * tid);
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        d[q] = make_float4(v[4 * q] * kRhtNorm, v[4 * q + 1] * kRhtNorm, v[4 * q + 2] * kRhtNorm,
-                           v[4 * q + 3] * kRhtNorm);
+      for (int i = 0; i < 16; ++i) xs[xs_pos<FMT>(16 * tid + i)] = v[i] * kRhtNorm;
     }
   } else if (tid < T::kWeights / 8) {
-    const uint32_t w[4] = {r.v0.x, r.v0.y, r.v0.z, r.v0.w};
-    float f[8];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      f[2 * q] = __uint_as_float(w[q] << 16);
-      f[2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
-    }
-    float4* d = reinterpret_cast<float4*>(xs + 8 * tid);
-    d[0] = make_float4(f[0], f[1], f[2], f[3]);
-    d[1] = make_float4(f[4], f[5], f[6], f[7]);
+    x_store8<FMT>(r.v0, xs, tid);
   }
 }
 
@@ -193,7 +203,7 @@ __device__ __forceinline__ void build_table(int nb, uint32_t tbase, const float*
   for (int e = 0; e < T::kDigits; ++e) {
     const int ka = digit_weight<FMT>(slot, l0, e, nb);
     const int kb = digit_weight<FMT>(slot, l0 + 1, e, nb);
-    xv[e] = make_float2(ka >= 0 ? xs[ka] : 0.0f, kb >= 0 ? xs[kb] : 0.0f);
+    xv[e] = make_float2(ka >= 0 ? xs[xs_pos<FMT>(ka)] : 0.0f, kb >= 0 ? xs[xs_pos<FMT>(kb)] : 0.0f);
   }
   const uint32_t col = tbase + (slot >> 1) * kPage + (slot & 1) * 128 + l0 * 4;
   constexpr int kStep = kThreadsT / 64;

@@ -222,7 +222,8 @@ lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const in
  * LBQ_ERR_ALIGN (p not 16-byte aligned), LBQ_ERR_CUDA. */
 lbq_status lbq_read_probe(const void* p, size_t bytes, uint32_t* sink, void* stream);
 
-/* Most products one launch of lbq_gemv_batch takes (longer lists run as several). */
+/* Most products one launch of lbq_gemv_batch takes (longer lists, or lists of several
+ * formats, run as several). */
 #define LBQ_BATCH_MAX 256
 
 /* One batch-1 product of a list: y = W_hat x (W_hat from w; D for LBQ_Q2RHT, else NULL). */
@@ -239,8 +240,11 @@ typedef struct lbq_product {
 size_t lbq_gemv_batch_workspace_bytes(const lbq_product* ps, int32_t n);
 
 /* n independent batch-1 products, each with the result lbq_gemv gives it, computed by
- * one persistent launch per LBQ_BATCH_MAX products ([tern] §1.2, [block] §2.1-2.2,
- * [sign], [rht]: the same lookup arithmetic as lbq_gemv). One CTA per SM stays
+ * one persistent launch per format present and LBQ_BATCH_MAX products of it ([tern]
+ * §1.2, [block] §2.1-2.2, [sign], [rht]: the same lookup arithmetic as lbq_gemv); a
+ * list of several formats runs format by format, in list order within a format (the
+ * kernel is compiled once per format: one that chose per product ran about twice as
+ * slowly, short of registers). One CTA per SM stays
  * resident for the whole list, so no product pays for a launch, a dependency wait or
  * a separate split-K kernel, and the weight stream runs on between products: while
  * the compute warps rebuild their lookup table for a product, a helper warp has the
