@@ -138,6 +138,31 @@ lbq_status lbq_cuda_status(cudaError_t e) {
   return LBQ_ERR_CUDA;
 }
 
+// The launches of a batch: the kernel runs one format a launch, so a list of several
+// runs as one launch (or chunk of LBQ_BATCH_MAX) per format present, in the list's
+// order within each format. fn(list, count) returns false to stop.
+template <typename F>
+void for_each_batch_launch(const lbq_product* ps, int32_t n, F fn) {
+  bool one_format = true;
+  for (int32_t i = 1; i < n; ++i) one_format = one_format && ps[i].w.fmt == ps[0].w.fmt;
+  std::vector<lbq_product> sub;
+  for (const int32_t fmt : {LBQ_TERN5, LBQ_SIGN1, LBQ_Q2RHT}) {
+    const lbq_product* list = ps;
+    int32_t count = n;
+    if (!one_format) {
+      sub.clear();
+      for (int32_t i = 0; i < n; ++i)
+        if (ps[i].w.fmt == fmt) sub.push_back(ps[i]);
+      list = sub.data();
+      count = static_cast<int32_t>(sub.size());
+    } else if (ps[0].w.fmt != fmt) {
+      continue;
+    }
+    for (int32_t i = 0; i < count; i += LBQ_BATCH_MAX)
+      if (!fn(list + i, count - i < LBQ_BATCH_MAX ? count - i : LBQ_BATCH_MAX)) return;
+  }
+}
+
 extern "C" {
 
 int32_t lbq_last_cuda_error(void) { return g_last_cuda_error; }
@@ -253,10 +278,11 @@ lbq_status lbq_gemv_f32(const lbq_weights* w, const uint16_t* x, const int8_t* D
 size_t lbq_gemv_batch_workspace_bytes(const lbq_product* ps, int32_t n) {
   if (check_batch(ps, n) != LBQ_OK) return 0;
   size_t need = 0;
-  for (int32_t i = 0; i < n; i += LBQ_BATCH_MAX) {
-    const size_t b = lbq_gemv_batch_ws(ps + i, n - i < LBQ_BATCH_MAX ? n - i : LBQ_BATCH_MAX);
+  for_each_batch_launch(ps, n, [&](const lbq_product* list, int32_t count) {
+    const size_t b = lbq_gemv_batch_ws(list, count);
     if (b > need) need = b;
-  }
+    return true;
+  });
   return need;
 }
 
@@ -267,33 +293,16 @@ lbq_status lbq_gemv_batch(const lbq_product* ps, int32_t n, void* workspace,
   const size_t need = lbq_gemv_batch_workspace_bytes(ps, n);
   if (!workspace || workspace_bytes < need) return LBQ_ERR_WORKSPACE;
   if (!aligned(workspace, 16)) return LBQ_ERR_ALIGN;
-  // The kernel runs one format a launch: a list of several runs as one launch (or
-  // chunk of LBQ_BATCH_MAX) per format present, in the list's order within each format.
-  bool one_format = true;
-  for (int32_t i = 1; i < n; ++i) one_format = one_format && ps[i].w.fmt == ps[0].w.fmt;
-  std::vector<lbq_product> sub;
-  for (const int32_t fmt : {LBQ_TERN5, LBQ_SIGN1, LBQ_Q2RHT}) {
-    const lbq_product* list = ps;
-    int32_t count = n;
-    if (!one_format) {
-      sub.clear();
-      for (int32_t i = 0; i < n; ++i)
-        if (ps[i].w.fmt == fmt) sub.push_back(ps[i]);
-      list = sub.data();
-      count = static_cast<int32_t>(sub.size());
-    } else if (ps[0].w.fmt != fmt) {
-      continue;
+  for_each_batch_launch(ps, n, [&](const lbq_product* list, int32_t count) {
+    const cudaError_t e = lbq_launch_gemv_batch(list, count, workspace, as_stream(stream));
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      st = lbq_cuda_status(e);
+      return false;
     }
-    for (int32_t i = 0; i < count; i += LBQ_BATCH_MAX) {
-      const cudaError_t e = lbq_launch_gemv_batch(
-          list + i, count - i < LBQ_BATCH_MAX ? count - i : LBQ_BATCH_MAX, workspace, as_stream(stream));
-      if (e != cudaSuccess) {
-        cudaGetLastError();
-        return lbq_cuda_status(e);
-      }
-    }
-  }
-  return LBQ_OK;
+    return true;
+  });
+  return st;
 }
 
 lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const int8_t* D,

@@ -1,29 +1,38 @@
-// gemv_batch.cu -- many independent batch-1 products in one persistent launch.
+// gemv_batch.cu -- many independent batch-1 products in one launch (stream-K schedule).
 //
 // The products are those of gemv.cu (ternary add/subtract/skip per block, pptc.cn
 // ternary-27B article §1.2 and mhpq.cn "27B in 5.9 GB" article §2.1-2.2; 1-bit Q1_0,
 // neodrop.ai round-up part 2; 2-bit with the rotated input, feinterview.poetries.top
 // "27B in 12 GB" article), computed with the same byte-lookup tables (lut.cuh). What
-// changes is how a list of them is scheduled: one CTA per SM stays resident for the
-// whole list, so nothing is paid per product for a launch, a dependency wait or a
-// split-K tail kernel, and the weight stream never stops between products.
+// changes is how a list of them is scheduled.
 //
-// Per CTA and product: one K-slice and a range of 16-row units (the same split as
-// the single-product kernel). Warps 0-14 load the x slice, build the 128 KB table,
-// then take units: each lane loads its word of four rows per group with 16-byte
-// global loads (no L1 allocation), one unit ahead, looks its bytes up, and the warp
-// reduces the unit's 16 rows with a transpose-reduce butterfly whose first stages
-// stay inside one scale block, so the block scales multiply 2 (ternary), 4 (1-bit)
-// or 8 (2-bit) values a lane instead of 16. Warp 15 (the helper) runs beside them:
-// it prefetches the next product's weights and x into L2 (bulk prefetch), so HBM keeps
-// streaming while the table is rebuilt, and it adds up the slice sums of the previous
-// product for its share of rows (split-K, in a fixed order: deterministic) once
-// every CTA has counted itself done with that product.
+// Work is counted in unit-slices: one 16-row unit of one K-slice (512 weights; 1024 for
+// the 1-bit format). A product of KS slices and NU units costs KS * NU. The list's
+// products are laid end to end, each as NU row-units of full K, and the total is cut
+// into one equal, contiguous range per CTA (one CTA per SM): every CTA computes whole
+// rows of one or a few products, all of K, so its rows need nobody else's sums. It
+// walks its range slice by slice: for each slice it builds the 128 KB lookup table of
+// that slice of x once and runs all its units of that product through it, keeping
+// each row's running sum in shared memory (in chunks of up to kAccUnits units), so a
+// table build serves hundreds of units. For a 64-layer pass each CTA builds about 20
+// tables, where a product-by-product split builds one per product (256).
 //
-// Synchronisation between CTAs is through counters at the start of the workspace
-// (done and reduced per product, and an exit count); the last CTA to leave resets
-// them, so every completed launch leaves them zero. The launch is cooperative, so
-// all CTAs are resident together, and every wait is bounded (fault code 12).
+// A product whose row-units are too coarse for that cut (few rows, many slices: a
+// CTA's share would be a fraction of one row-unit) is split along K into S pieces
+// of consecutive slices; each piece writes its fp32 sums to the workspace and a small
+// second kernel adds the S pieces of every row in a fixed order (deterministic). The
+// rule is on the host (pieces_for); a 27B-layer pass has no split product.
+//
+// There is no communication between CTAs at all: no counters, no waits. Inside a CTA,
+// 16 warps build the table together (two barriers per slice), then take units: each
+// lane loads its word of four rows per group with 16-byte global loads (no L1
+// allocation, evict-first in L2), one unit ahead, looks its bytes up, and the warp
+// reduces the unit's 16 rows with the butterfly of lut.cuh. The next slice's x comes
+// in by cp.async while the units run, and each warp's first two units of the next
+// slice are loaded before its table is built, so the weight stream runs on through
+// the build.
+#include <vector>
+
 #include "lut.cuh"
 #include "sm100_async.cuh"
 
@@ -32,80 +41,64 @@ namespace {
 using namespace lbq;
 using namespace lbq::lut;
 
-// The SM's register file is split between its four schedulers: a CTA of 16 warps (four
-// per scheduler) may use 128 registers a thread, one of 17 to 20 warps only 96.
-#ifndef LBQ_BATCH_WARPS
-#define LBQ_BATCH_WARPS 15
-#endif
-constexpr int kCWarps = LBQ_BATCH_WARPS;     // compute warps
-constexpr int kCThreads = 32 * kCWarps;      // compute threads
-constexpr int kBuildThreads = kCThreads / 64 * 64;  // the table build takes whole column sets of 64
-constexpr int kMaxRegs = kCWarps + 1 <= 16 ? 128 : 96;
-constexpr int kBThreads = kCThreads + 32;    // + the helper warp
-constexpr int kRows = 16;                    // rows per unit (four groups of four)
-constexpr int kLag = 4;                      // a product's split-K sum waits this many products
-// Partial-sum buffers in flight. Product p's buffer was last used by p - kRing, summed
-// during p - kRing + kLag; the helper checks that sum while readying p, two products
-// ahead of the compute warps, having released its own CTA's sums up to p - 3: so
-// p - kRing + kLag <= p - 3 at least; three products more leave slack for CTAs that
-// run behind.
-#ifndef LBQ_BATCH_RING_SLACK
-#define LBQ_BATCH_RING_SLACK 3
-#endif
-constexpr int kRing = kLag + 3 + LBQ_BATCH_RING_SLACK;
-// The helper asks L2 for the first kPrefetchUnits units of each compute warp of a
-// product while the warps build its table (the warps' own loads then run a unit ahead:
-// prefetches of their own measured no faster).
-constexpr int kPrefetchUnits = 4;
-#ifndef LBQ_BATCH_HELPER_PREFETCH
-#define LBQ_BATCH_HELPER_PREFETCH 0
-#endif
-constexpr uint32_t kXBytes = lut::kXsBytes;  // one padded x slice as fp32
-constexpr int kXBufs = 3;                    // x slices in shared memory (the helper works 2 ahead)
-constexpr uint32_t kMiscBytes = kXBufs * kXBytes + 1024;  // x slices, flags
-constexpr uint32_t kDescSmem = 16384;        // the product list, copied to shared memory
-constexpr uint32_t kSmemBatch = 192 * 1024;  // the table needs a 64 KB-aligned 128 KB
-constexpr unsigned kFaultBatch = 12, kFaultBatchLayout = 13;
+// 16 warps (four per scheduler) may use 128 registers a thread.
+constexpr int kWarps = 16;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kRows = 16;  // rows per unit (four groups of four)
+// Units a chunk keeps running sums for in shared memory (a multiple of kWarps): 63 KB,
+// the room below a 64 KB-aligned table when the dynamic window starts 1 KB in.
+constexpr int32_t kAccUnits = 1008;
+constexpr uint32_t kAccBytes = kAccUnits * kRows * 4;
+// The split rule: one row-unit of a piece may cost at most 1 / kMinUnitsPerTable of a
+// CTA's share, so that a table build serves at least that many units.
+constexpr int64_t kMinUnitsPerTable = 64;
+constexpr uint32_t kXRawBytes = 2048;  // one x slice as bf16 (1024 weights at most)
+constexpr uint32_t kDRawBytes = 512;   // its rotation signs (2-bit format)
+constexpr uint32_t kMiscBytes = kXRawBytes + kDRawBytes + kXsBytes + 64;  // + the start index
+constexpr uint32_t kSmemBatch = 227 * 1024;
+constexpr unsigned kFaultBatchLayout = 13;
 constexpr int kMaxBatch = LBQ_BATCH_MAX;
-// counters (32-bit words at the start of the workspace)
-constexpr int kCtrDone = 0, kCtrReduced = kMaxBatch, kCtrExit = 2 * kMaxBatch;
 
-// One product as the kernel sees it (64 bytes). The list lives in the workspace, after
-// the counters, written there by the install kernel before each launch: the main
-// kernel's own parameters stay small.
+static_assert(kAccUnits % kWarps == 0, "chunks are whole rounds of units");
+static_assert(kAccBytes <= 63 * 1024, "the sums fit below the table");
+
+// One product as the kernel sees it (80 bytes), written into the workspace by the
+// install kernel before each launch.
 struct __align__(16) BProd {
   const uint8_t* codes;
   const uint16_t* scales;
   const uint16_t* x;
   const int8_t* D;
   uint16_t* y;
+  int64_t c0;       // unit-slices of the products before this one
+  int64_t poff;     // first float of this product's piece sums (S > 1)
   int32_t cstride;  // code bytes per row
   int32_t sstride;  // fp16 scales per row
   int32_t N;
+  int32_t NU;       // 16-row units
   int16_t fmt;
   int16_t KS;       // K-slices
-  int16_t G;        // CTAs per slice
+  int16_t S;        // pieces along K (1: rows are whole on one CTA)
   int16_t nblk;     // scale blocks per row
 };
-static_assert(sizeof(BProd) == 64, "descriptor size");
-static_assert(LBQ_BATCH_MAX * sizeof(BProd) <= 16384, "the list fits its shared-memory copy");
-constexpr int kInstallChunk = 56;  // descriptors per install launch (parameters < 4 KB)
-constexpr size_t kDescBytes = kMaxBatch * sizeof(BProd);  // the list, after the ring buffers
+static_assert(sizeof(BProd) == 80, "descriptor size");
+constexpr int kInstallChunk = 48;  // descriptors per install launch (parameters < 4 KB)
+constexpr size_t kDescBytes = kMaxBatch * sizeof(BProd);
 
 struct BInstall {
   int32_t first, count;
   BProd* dst;
   BProd p[kInstallChunk];
 };
+static_assert(sizeof(BInstall) <= 4096, "install parameters");
 
 struct BArgs {
+  const BProd* p;   // the list (in the workspace)
+  float* partial;   // piece sums of split products
+  unsigned* fault;
+  int64_t W;        // unit-slices of the whole list
   int32_t n;
   int32_t pad;
-  int64_t ring_floats;  // floats per partial-sum buffer
-  float* ring;          // kRing buffers
-  unsigned* ctr;
-  unsigned* fault;
-  const BProd* p;       // the list (in the workspace)
 };
 
 __global__ void install_kernel(const __grid_constant__ BInstall in) {
@@ -113,40 +106,7 @@ __global__ void install_kernel(const __grid_constant__ BInstall in) {
   if (i < in.count) in.dst[in.first + i] = in.p[i];
 }
 
-// Adds v to a counter with release semantics at GPU scope: this thread's earlier writes,
-// and those of the threads that met it at a barrier just before, are visible to any
-// thread that then reads the new count with acquire semantics.
-__device__ __forceinline__ void red_release(unsigned* p, unsigned v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Spins (sleeping between polls) until *p >= target; gives up after the wait limit,
-// recording the fault code, or once another wait has given up.
-__device__ __forceinline__ bool wait_count(const unsigned* p, unsigned target, unsigned* fault) {
-  if (ld_acquire(p) >= target) return true;
-  const uint64_t t0 = global_ns();
-  for (uint32_t i = 1;; ++i) {
-    __nanosleep(i < 64 ? 32 : 256);
-    if (ld_acquire(p) >= target) return true;
-    if ((i & 63) == 0) {
-      if (*reinterpret_cast<volatile unsigned*>(fault) != 0) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
-        atomicExch(fault, kFaultBatch);
-        return false;
-      }
-    }
-  }
-}
-
-// Weight loads: read once, so they neither allocate in L1 nor stay in L2 for long
-// (an evict-first cache policy: the L2 keeps the prefetched weights of the next
-// product and the slice sums instead).
+// Weight loads: read once, so they neither allocate in L1 nor stay in L2 for long.
 __device__ __forceinline__ uint64_t evict_first_policy() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
@@ -166,36 +126,124 @@ __device__ __forceinline__ uint2 ldg_stream2(const void* p, uint64_t pol) {
                : "l"(p), "l"(pol));
   return v;
 }
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// The CTA's work on one product: virtual CTA v in [0, KS * G) is slice v / G and the
-// v % G-th share of the 16-row units.
-struct Part {
-  int32_t j, u_lo, u_hi, nb;
+// One step of a CTA's walk: slice j of the chunk [c0, c1) of this CTA's units [u0, u1)
+// of piece s (slices [j0, j1)) of product p; p < 0 when the walk is over.
+struct Seg {
+  int32_t p, s;
+  int32_t u0, u1;
+  int32_t c0, c1;
+  int32_t j, j0, j1;
 };
-template <int FMT>
-__device__ __forceinline__ Part part_of(const BProd& P, int v) {
-  using T = Traits<FMT>;
-  Part r;
-  const int32_t NU = (P.N + kRows - 1) / kRows;
-  r.j = v / P.G;
-  const int32_t gs = v - r.j * P.G;
-  r.u_lo = static_cast<int32_t>(static_cast<int64_t>(gs) * NU / P.G);
-  r.u_hi = static_cast<int32_t>(static_cast<int64_t>(gs + 1) * NU / P.G);
-  const int blk0 = r.j * T::kBlocks;
-  r.nb = P.nblk - blk0 < T::kBlocks ? P.nblk - blk0 : T::kBlocks;
-  return r;
+
+// Piece s of a product: slices [KS s / S, KS (s + 1) / S).
+__device__ __forceinline__ int32_t piece_start(int32_t KS, int32_t S, int32_t s) {
+  return static_cast<int32_t>(static_cast<int64_t>(KS) * s / S);
 }
 
-// Where this lane's loads of one warp's units are: copied into registers once per
-// product and slice, so that the stores of the unit loop cannot make the compiler
-// re-read the descriptor. Unit t of the warp is unit u0 + kCWarps t; its groups start
-// at w + t * ustep (+ q * gstride for group q); `ng` counts its groups that exist (the
-// matrix's last unit may reach past N).
+// The first piece at or after (p, s) with units in [lo, hi): unit u of piece s covers
+// the unit-slices [base + u len, base + (u + 1) len), base = c0 + NU j0, len = j1 - j0,
+// and belongs to the CTA whose range holds its first one.
+__device__ Seg find_piece(const BProd* list, int32_t n, int32_t p, int32_t s, int64_t lo, int64_t hi) {
+  Seg g;
+  g.p = -1;
+  for (; p < n; ++p, s = 0) {
+    const BProd& P = list[p];
+    if (P.c0 >= hi) return g;
+    for (; s < P.S; ++s) {
+      const int32_t j0 = piece_start(P.KS, P.S, s), j1 = piece_start(P.KS, P.S, s + 1);
+      const int64_t len = j1 - j0;
+      const int64_t base = P.c0 + static_cast<int64_t>(P.NU) * j0;
+      if (base >= hi) return g;
+      const int64_t u0 = lo > base ? (lo - base + len - 1) / len : 0;
+      int64_t u1 = (hi - base + len - 1) / len;
+      if (u1 > P.NU) u1 = P.NU;
+      if (u0 < u1) {
+        g.p = p;
+        g.s = s;
+        g.u0 = static_cast<int32_t>(u0);
+        g.u1 = static_cast<int32_t>(u1);
+        g.c0 = g.u0;
+        g.c1 = g.u1 - g.u0 > kAccUnits ? g.u0 + kAccUnits : g.u1;
+        g.j = g.j0 = j0;
+        g.j1 = j1;
+        return g;
+      }
+    }
+  }
+  return g;
+}
+
+__device__ __forceinline__ Seg advance(const BProd* list, int32_t n, Seg g, int64_t lo, int64_t hi) {
+  if (g.j + 1 < g.j1) {
+    ++g.j;
+    return g;
+  }
+  if (g.c1 < g.u1) {
+    g.c0 = g.c1;
+    g.c1 = g.u1 - g.c0 > kAccUnits ? g.c0 + kAccUnits : g.u1;
+    g.j = g.j0;
+    return g;
+  }
+  return find_piece(list, n, g.p, g.s + 1, lo, hi);
+}
+
+template <int FMT>
+__device__ __forceinline__ int blocks_in(const BProd& P, int32_t j) {
+  const int left = P.nblk - j * Traits<FMT>::kBlocks;
+  return left < Traits<FMT>::kBlocks ? left : Traits<FMT>::kBlocks;
+}
+
+// x slice j of P (and its signs) into the staging buffers, 16 bytes a thread by
+// cp.async (x and D are 16-byte aligned, slices start at 16-byte multiples).
+template <int FMT>
+__device__ __forceinline__ void x_fetch(const BProd& P, int32_t j, int nb, uint32_t xraw, uint32_t draw, int tid) {
+  using T = Traits<FMT>;
+  const int64_t k0 = static_cast<int64_t>(j) * T::kWeights;
+  if (FMT == LBQ_Q2RHT) {
+    if (tid < 32) {  // 16 activations and 16 signs a lane, as x_store rotates them
+      cp_async16(xraw + 32 * tid, P.x + k0 + 16 * tid);
+      cp_async16(xraw + 32 * tid + 16, P.x + k0 + 16 * tid + 8);
+      cp_async16(draw + 16 * tid, P.D + k0 + 16 * tid);
+    }
+  } else if (tid < T::kWeights / 8 && 8 * tid < nb * kTernBlock) {
+    cp_async16(xraw + 16 * tid, P.x + k0 + 8 * tid);
+  }
+  cp_async_commit();
+}
+
+// The staged slice as padded fp32 in xs (each thread converts what it fetched).
+template <int FMT>
+__device__ __forceinline__ void x_convert(int nb, uint32_t xraw, uint32_t draw, float* xs, int tid) {
+  using T = Traits<FMT>;
+  cp_async_wait_all();
+  if (FMT == LBQ_Q2RHT) {
+    if (tid < 32) {
+      XLoad r;
+      r.v0 = lds_v4(xraw + 32 * tid);
+      r.v1 = lds_v4(xraw + 32 * tid + 16);
+      r.d = lds_v4(draw + 16 * tid);
+      x_store<FMT>(r, xs, tid);
+    }
+  } else if (tid < T::kWeights / 8) {
+    const uint4 v = 8 * tid < nb * kTernBlock ? lds_v4(xraw + 16 * tid) : make_uint4(0u, 0u, 0u, 0u);
+    x_store8<FMT>(v, xs, tid);
+  }
+}
+
+// Where this lane's loads of one warp's units are, in registers for the unit loop.
+// Unit t of the warp is unit u0 + kWarps t; its groups start at w + t * ustep
+// (+ q * gstride for group q); `ng` counts the matrix's groups (its last unit may
+// reach past N).
 struct Stream {
   const uint8_t* w;   // this lane's word in group 0 of the warp's first unit
   const uint8_t* s;   // this lane's scale load for that unit
-  const uint8_t* s0;  // the slice's scale run of group 0 of that unit (1-bit, 2-bit)
-  uint32_t ustep;     // bytes between the warp's consecutive units (15 units apart)
+  uint32_t ustep;     // bytes between the warp's consecutive units (kWarps units apart)
   uint32_t sustep;    // the same for the scale loads
   uint32_t gstride;   // code bytes per group of four rows
   uint32_t sstep;     // scale bytes between consecutive groups (1-bit, 2-bit)
@@ -204,43 +252,40 @@ struct Stream {
 };
 
 template <int FMT>
-__device__ __forceinline__ Stream make_stream(const BProd& P, const Part& pt, int32_t u0, int lane,
+__device__ __forceinline__ Stream make_stream(const BProd& P, int32_t j, int nb, int32_t u0, int lane,
                                               uint32_t woff) {
   using T = Traits<FMT>;
   Stream st;
   st.gstride = 4u * static_cast<uint32_t>(P.cstride);
-  st.ustep = kCWarps * 4u * st.gstride;
+  st.ustep = kWarps * 4u * st.gstride;
   st.ng = (P.N + 3) / 4;
   st.g0 = 4 * u0;
-  st.w = P.codes + static_cast<int64_t>(st.g0) * st.gstride + pt.j * T::kGroupBytes + woff;
+  st.w = P.codes + static_cast<int64_t>(st.g0) * st.gstride + j * T::kGroupBytes + woff;
   if (FMT == LBQ_TERN5) {
     // rows R, R + 1 after three butterfly stages (R = 8 b0 + 4 b1 + 2 b2 of the lane)
     const int R = 8 * (lane & 1) + 4 * ((lane >> 1) & 1) + 2 * ((lane >> 2) & 1);
     int b = lane >> 3;
-    if (b >= pt.nb) b = pt.nb - 1;  // no block here: any finite scale times a zero sum
-    st.s = P.codes + static_cast<int64_t>(st.g0 + (R >> 2)) * st.gstride +
-           16 * (pt.j * T::kWords + 7 * b + 6) + 4 * (R & 3);
-    st.s0 = st.s;
+    if (b >= nb) b = nb - 1;  // no block here: any finite scale times a zero sum
+    st.s = P.codes + static_cast<int64_t>(st.g0 + (R >> 2)) * st.gstride + 16 * (j * T::kWords + 7 * b + 6) +
+           4 * (R & 3);
     st.sstep = 0;
     st.sustep = st.ustep;
   } else {
     st.sstep = 8u * static_cast<uint32_t>(P.sstride);  // scale bytes per group of four rows
-    st.sustep = kCWarps * 4u * st.sstep;
+    st.sustep = kWarps * 4u * st.sstep;
     const int b = FMT == LBQ_SIGN1 ? (lane >> 2) : (lane >> 1);
-    const int bb = b < pt.nb ? b : pt.nb - 1;
+    const int bb = b < nb ? b : nb - 1;
     const int gl = FMT == LBQ_SIGN1 ? 2 * (lane & 1) + ((lane >> 1) & 1) : 2 * (lane & 1);
-    st.s0 = reinterpret_cast<const uint8_t*>(P.scales) + static_cast<int64_t>(st.g0) * st.sstep +
-            pt.j * T::kScaleBytes;
-    st.s = st.s0 + gl * st.sstep + 8 * bb;
+    st.s = reinterpret_cast<const uint8_t*>(P.scales) + static_cast<int64_t>(st.g0) * st.sstep +
+           j * T::kScaleBytes + gl * st.sstep + 8 * bb;
   }
   return st;
 }
 
 template <int FMT>
-__device__ __forceinline__ void load_unit(const Stream& st, int32_t t, int lane, uint64_t pol,
-                                          UnitRegs& r) {
+__device__ __forceinline__ void load_unit(const Stream& st, int32_t t, int lane, uint64_t pol, UnitRegs& r) {
   const uint8_t* w = st.w + static_cast<uint64_t>(t) * st.ustep;
-  const int32_t left = st.ng - (st.g0 + 4 * kCWarps * t);  // groups of this unit that exist
+  const int32_t left = st.ng - (st.g0 + 4 * kWarps * t);  // groups of this unit that exist
   if (left >= 4) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) r.w[q] = ldg_stream(w + q * st.gstride, pol);
@@ -262,451 +307,130 @@ __device__ __forceinline__ void load_unit(const Stream& st, int32_t t, int lane,
   }
 }
 
-// Asks L2 for a line (a hint: later loads find it in L2 instead of waiting on HBM).
-__device__ __forceinline__ void prefetch_line(const void* p) {
-  asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
-}
-
-
-// The deferred split-K sum of one product for this CTA's share of its rows, done by the
-// compute warps two products later (every CTA is then long done with it): the loads
-// are issued before the table build, whose shared-memory work hides their latency,
-// and finished after it. Row r of the share is summed by P consecutive threads, each
-// over a run of at most kRun slices, combined by a fixed shuffle tree (deterministic).
-constexpr int kRun = 8;
-
-// This CTA's split-K sum of one product: rows [n0, n1), logP: log2 of the threads a row
-// (2^logP runs of at most kRun slices each). Computed once per product (divisions are
-// slow) by the helper, or by reduce_plan in the tail.
-struct RedPlan {
-  int32_t n0, n1, logP, run;
-};
-__device__ __forceinline__ RedPlan reduce_plan(const BProd& P) {
-  RedPlan rp;
-  rp.logP = 0;
-  while ((P.KS + (1 << rp.logP) - 1) >> rp.logP > kRun) ++rp.logP;  // at most 64 threads a row
-  rp.run = (P.KS + (1 << rp.logP) - 1) >> rp.logP;
-  rp.n0 = static_cast<int32_t>(static_cast<int64_t>(blockIdx.x) * P.N / gridDim.x);
-  rp.n1 = static_cast<int32_t>(static_cast<int64_t>(blockIdx.x + 1) * P.N / gridDim.x);
-  return rp;
-}
-
-struct Reduce {
-  float v[kRun];
-  int32_t row;   // this thread's row, or -1
-  int32_t nv;    // slices in its run
-};
-
-__device__ __forceinline__ void reduce_begin(const BArgs& a, int q, const RedPlan& rp, int tid, int batch,
-                                             Reduce& r) {
-  const BProd& P = a.p[q];
-  const int rows_per_batch = kCThreads >> rp.logP;
-  const int32_t row = rp.n0 + batch * rows_per_batch + (tid >> rp.logP);
-  const int sub = tid & ((1 << rp.logP) - 1);
-  r.row = -1;
-  r.nv = 0;
-#pragma unroll
-  for (int i = 0; i < kRun; ++i) r.v[i] = 0.0f;
-  if (tid < (rows_per_batch << rp.logP) && row < rp.n1) {
-    r.row = row;
-    const int j0 = sub * rp.run;
-    r.nv = P.KS - j0 < rp.run ? (P.KS - j0 > 0 ? P.KS - j0 : 0) : rp.run;
-    const float* part = a.ring + static_cast<int64_t>(q % kRing) * a.ring_floats + row;
-    // predicated loads into zeroed registers: nothing waits for them until reduce_end
-#pragma unroll
-    for (int i = 0; i < kRun; ++i)
-      asm volatile(
-          "{\n\t.reg .pred p;\n\tsetp.lt.s32 p, %2, %3;\n\t@p ld.global.cg.f32 %0, [%1];\n\t}"
-          : "+f"(r.v[i])
-          : "l"(part + static_cast<int64_t>(j0 + i) * P.N), "r"(i), "r"(r.nv));
-  }
-}
-
-// Adds the loaded runs, combines each row's runs (fixed shuffle tree), stores y; returns
-// whether rows remain for another batch.
-__device__ __forceinline__ bool reduce_end(const BArgs& a, int q, const RedPlan& rp, int tid, int batch,
-                                           Reduce& r) {
-  const BProd& P = a.p[q];
-  float s = 0.0f;
-#pragma unroll
-  for (int i = 0; i < kRun; ++i)
-    if (i < r.nv) s += r.v[i];
-  const int np = 1 << rp.logP;
-  for (int o = 1; o < np; o <<= 1) s += __shfl_down_sync(0xffffffffu, s, o, np);
-  if (r.row >= 0 && (tid & (np - 1)) == 0) P.y[r.row] = f32_to_bf16_bits(s);
-  return rp.n0 + (batch + 1) * (kCThreads >> rp.logP) < rp.n1;
-}
-
-// The whole share of product q at once (no table build to hide behind).
-__device__ __forceinline__ void reduce_all(const BArgs& a, int q, int tid) {
-  const RedPlan rp = reduce_plan(a.p[q]);
-  Reduce r;
-  for (int batch = 0;; ++batch) {
-    reduce_begin(a, q, rp, tid, batch, r);
-    if (!reduce_end(a, q, rp, tid, batch, r)) break;
-  }
-}
-
-// What the helper works out for the compute warps while readying product p: the
-// first share of p this CTA takes and the split-K sum of p - kLag it adds.
-struct Prep {
-  Part pt;
-  RedPlan rp;
-};
-
-// The x slice of this CTA's first share of product p (slice j), converted to fp32 (the
-// 2-bit format: rotated) into xs by one warp; the helper does this a product ahead.
+// The lane's word offset within a group's slice run (lanes without a word read a
+// neighbour's: their table entries are zero-weight columns).
 template <int FMT>
-__device__ __forceinline__ void x_slice_warp(const BProd& P, int32_t j, int nb, float* xs, int lane) {
-  using T = Traits<FMT>;
-  if (FMT == LBQ_Q2RHT) {
-    x_store<FMT>(x_issue<FMT>(P.x, P.D, P.nblk, j, lane), xs, lane);
-  } else {
-    const uint4* x8 = reinterpret_cast<const uint4*>(P.x + static_cast<int64_t>(j) * T::kWeights);
-    constexpr int kChunks = T::kWeights / 8;  // 16-byte chunks of 8 activations
-    uint4 v[kChunks / 32];
-#pragma unroll
-    for (int i = 0; i < kChunks / 32; ++i) {
-      const int c = lane + 32 * i;
-      v[i] = 8 * c < nb * kTernBlock ? __ldg(x8 + c) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int i = 0; i < kChunks / 32; ++i) x_store8<FMT>(v[i], xs, lane + 32 * i);
-  }
-}
-
-// Shared-memory flags between the compute warps and the helper (CTA scope).
-struct Flags {
-  int started;    // products the compute warps have started
-  int built;      // products whose table the compute warps have built
-  int gate;       // products < gate may start: x slice in place, global counters checked
-  int unitsdone;  // products whose units (and the sum due with them) the compute warps finished
-};
-__device__ __forceinline__ void st_release_cta(volatile int* p, int v) {
-  asm volatile("st.release.cta.shared.u32 [%0], %1;" ::"r"(smem_u32(const_cast<int*>(p))), "r"(v) : "memory");
-}
-__device__ __forceinline__ int ld_acquire_cta(const volatile int* p) {
-  int v;
-  asm volatile("ld.acquire.cta.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(const_cast<int*>(p))) : "memory");
-  return v;
-}
-
-// Spins on a shared-memory counter written by another warp of the CTA; gives up after
-// the wait limit, recording the fault code, or as soon as any wait has given up.
-__device__ __forceinline__ bool wait_smem(const volatile int* c, int target, unsigned* fault) {
-  if (ld_acquire_cta(c) >= target) return true;
-  const uint64_t t0 = global_ns();
-  for (uint32_t i = 1; ld_acquire_cta(c) < target; ++i) {
-    __nanosleep(32);
-    if ((i & 63) == 0) {
-      if (*reinterpret_cast<volatile unsigned*>(fault) != 0) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
-        atomicExch(fault, kFaultBatch);
-        return false;
-      }
-    }
-  }
-  return true;
+__device__ __forceinline__ uint32_t word_offset(int lane, int nb) {
+  const int wl = lane_word<FMT>(lane, nb);
+  const int wq = lane_word<FMT>(lane & ~7, nb);
+  return 16u * static_cast<uint32_t>(wl >= 0 ? wl : (wq >= 0 ? wq : 0));
 }
 
 template <int FMT>
-__device__ __forceinline__ void compute_product(const BArgs& a, int p, uint32_t tbase, float* xbuf,
-                                                volatile Flags* fl, const Prep* prep, int tid, bool& ok) {
-  using T = Traits<FMT>;
-  const BProd& P = a.p[p];
-  const int warp = tid >> 5, lane = tid & 31;
-  const int participants = P.KS * P.G;
-  float* part = a.ring + static_cast<int64_t>(p % kRing) * a.ring_floats;
-  float* const xs = xbuf + (p % kXBufs) * (kXBytes / 4);
-  // The helper opens the gate of product p once its x slice is in xs, every CTA is done
-  // with product q = p - kLag (whose split-K sum is added here) and every CTA has summed
-  // product p - kRing (the last user of the ring buffer this product writes).
-  const int q = p - kLag;
-  const bool red = q >= 0 && a.p[q].KS > 1;
-  if (tid == 0 && ok) ok = wait_smem(&fl->gate, p + 1, a.fault);
-  named_bar_sync(1, kCThreads);
-  // a CTA with no share of this product has no table to build: nothing to wait for
-  if (tid == 0 && static_cast<int>(blockIdx.x) >= participants) st_release_cta(&fl->built, p + 1);
-  const Prep& pr = prep[p % kXBufs];  // written by the helper before it opened the gate
-  const RedPlan rp = pr.rp;
-  Reduce r;
-  bool rmore = false;
-  if (red) reduce_begin(a, q, rp, tid, 0, r);
-  bool rpending = red;
-  bool first = true;
-  for (int v = blockIdx.x; v < participants; v += gridDim.x) {
-    const Part pt = first ? pr.pt : part_of<FMT>(P, v);
-    if (!first) {  // a further share of this product (more slices than CTAs)
-      x_store<FMT>(x_issue<FMT>(P.x, P.D, P.nblk, pt.j, tid), xs, tid);
-      named_bar_sync(1, kCThreads);
-    }
-    first = false;
-    if (tid < kBuildThreads) build_table<FMT, kBuildThreads>(pt.nb, tbase, xs, tid);
-    if (rpending) {  // the sum's loads have landed behind the build
-      rmore = reduce_end(a, q, rp, tid, 0, r);
-      rpending = false;
-    }
-    named_bar_sync(1, kCThreads);
-    if (tid == 0) st_release_cta(&fl->built, p + 1);
-
-    const int wl = lane_word<FMT>(lane, pt.nb);
-    const int wq = lane_word<FMT>(lane & ~7, pt.nb);
-    const uint32_t woff = 16u * static_cast<uint32_t>(wl >= 0 ? wl : (wq >= 0 ? wq : 0));
-    const uint32_t lanereg = tbase | static_cast<uint32_t>(lane * 4);
-    const int rloc = 8 * (lane & 1) + 4 * ((lane >> 1) & 1) + 2 * ((lane >> 2) & 1) + ((lane >> 3) & 1);
-    const int32_t n_units = pt.u_hi - pt.u_lo;
-    const int32_t nt = n_units > warp ? (n_units - warp + kCWarps - 1) / kCWarps : 0;
-    // the row this lane stores for the warp's unit t: row0 + 16 kCWarps t
-    const int32_t N = P.N;
-    const int32_t row0 = (pt.u_lo + warp) * kRows + rloc;
-    const bool store_lane = lane < 16;
-    uint16_t* const yp = P.y;
-    float* const part_j = part + static_cast<int64_t>(pt.j) * N;
-    const bool direct = P.KS == 1;
-    const Stream st = make_stream<FMT>(P, pt, pt.u_lo + warp, lane, woff);
-    const uint64_t pol = evict_first_policy();
-    auto finish = [&](float val, int32_t t) {
-      const int32_t row = row0 + kRows * kCWarps * t;
-      if (store_lane && row < N) {
-        if (direct) yp[row] = f32_to_bf16_bits(val);
-        else part_j[row] = val;
-      }
-    };
-    // two register buffers, one unit's loads in flight while the other is looked up
-    // (a third measured no faster); unrolled by two so that they swap without copies
-    UnitRegs ra, rb;
-    if (nt > 0) load_unit<FMT>(st, 0, lane, pol, ra);
-    for (int32_t t = 0; t < nt; t += 2) {
-      if (t + 1 < nt) load_unit<FMT>(st, t + 1, lane, pol, rb);
-      finish(unit_sum<FMT>(ra, lanereg, lane), t);
-      if (t + 1 >= nt) break;
-      if (t + 2 < nt) load_unit<FMT>(st, t + 2, lane, pol, ra);
-      finish(unit_sum<FMT>(rb, lanereg, lane), t + 1);
-    }
-    named_bar_sync(1, kCThreads);  // every warp is done with the table
-  }
-  if (rpending) rmore = reduce_end(a, q, rp, tid, 0, r);  // this CTA had no share of product p
-  if (red && rmore) {  // a share larger than one batch: the rest, without overlap
-    for (int rbatch = 1;; ++rbatch) {
-      reduce_begin(a, q, rp, tid, rbatch, r);
-      if (!reduce_end(a, q, rp, tid, rbatch, r)) break;
-    }
-  }
-  // the slice sums of p and the sums of q are stored: the helper releases them
-  named_bar_sync(1, kCThreads);
-  if (tid == 0) st_release_cta(&fl->unitsdone, p + 1);
-}
-
-// The last products' sums, after the compute warps' final product (the helper has
-// checked that every CTA is done with them).
-__device__ __forceinline__ void reduce_tail(const BArgs& a, volatile Flags* fl, int tid, bool& ok) {
-  if (tid == 0 && ok) ok = wait_smem(&fl->gate, a.n + 1, a.fault);
-  named_bar_sync(1, kCThreads);
-  for (int q = a.n - kLag > 0 ? a.n - kLag : 0; q < a.n; ++q)
-    if (a.p[q].KS > 1) reduce_all(a, q, tid);
-}
-
-// The helper's L2 prefetch of the first units of each of this CTA's warps for product p
-// (kPrefetchUnits of them, as the warps' own prefetch runs that far ahead), so that HBM
-// keeps streaming while the compute warps build the product's table.
-template <int FMT>
-__device__ __forceinline__ void prefetch_product(const BArgs& a, int p, int lane) {
-  using T = Traits<FMT>;
-  const BProd& P = a.p[p];
-  const int participants = P.KS * P.G;
-  const int32_t NG = (P.N + 3) / 4;
-  for (int v = blockIdx.x; v < participants; v += gridDim.x) {
-    const Part pt = part_of<FMT>(P, v);
-    const uint32_t cbytes = FMT == LBQ_TERN5 ? 112u * pt.nb : (FMT == LBQ_SIGN1 ? 64u * pt.nb : 512u);
-    const int32_t g0 = 4 * pt.u_lo;
-    int32_t g1 = 4 * (pt.u_lo + kCWarps * (kPrefetchUnits + 1));
-    if (g1 > 4 * pt.u_hi) g1 = 4 * pt.u_hi;
-    if (g1 > NG) g1 = NG;
-    const uint8_t* base = P.codes + pt.j * T::kGroupBytes;
-    const int64_t gstride = 4 * static_cast<int64_t>(P.cstride);
-    // each group's run, line by line (128-byte lines; runs of 448 or 512 bytes)
-    const int lines = static_cast<int>((cbytes + 127) / 128) + 1;
-    for (int32_t i = lane; i < (g1 - g0) * lines; i += 32) {
-      const int32_t g = g0 + i / lines;
-      const uint32_t off = 128u * static_cast<uint32_t>(i % lines);
-      if (off < cbytes + 127) prefetch_line(base + g * gstride + (off < cbytes ? off : cbytes - 1));
-    }
-    if (FMT != LBQ_TERN5) {
-      const uint8_t* sb = reinterpret_cast<const uint8_t*>(P.scales) + pt.j * T::kScaleBytes;
-      for (int32_t g = g0 + lane; g < g1; g += 32) prefetch_line(sb + g * 8 * static_cast<int64_t>(P.sstride));
-    }
-  }
-}
-
-// The helper's preload of the x slice of this CTA's first share of product p.
-template <int FMT>
-__device__ __forceinline__ void xload_product(const BArgs& a, int p, float* xs, int lane) {
-  const BProd& P = a.p[p];
-  if (static_cast<int>(blockIdx.x) < P.KS * P.G) {
-    const Part pt = part_of<FMT>(P, blockIdx.x);
-    x_slice_warp<FMT>(P, pt.j, pt.nb, xs, lane);
-  }
-}
-
-// Format masks: the kernel is compiled once per set of formats a list holds, so that a
-// list of one format gets code (and registers) for that format alone.
-// The kernel is compiled once per format (kFmts = that format's bit): one kernel that
-// chose the format per product needed more registers than a thread has, and ran every
-// phase of a pass about twice as slowly (measured on a ternary list, as a function
-// call per product and inlined alike), so a list of several formats is run as one
-// launch per format (the products are independent).
-__host__ __device__ constexpr int fmt_bit(int fmt) { return 1 << (fmt - 1); }
-
-template <int kFmts>
-__device__ __forceinline__ void prefetch_any(const BArgs& a, int p, int lane) {
-  const int f = a.p[p].fmt;
-  if ((kFmts & fmt_bit(LBQ_TERN5)) && f == LBQ_TERN5) prefetch_product<LBQ_TERN5>(a, p, lane);
-  if ((kFmts & fmt_bit(LBQ_SIGN1)) && f == LBQ_SIGN1) prefetch_product<LBQ_SIGN1>(a, p, lane);
-  if ((kFmts & fmt_bit(LBQ_Q2RHT)) && f == LBQ_Q2RHT) prefetch_product<LBQ_Q2RHT>(a, p, lane);
-}
-template <int kFmts>
-__device__ __forceinline__ void xload_any(const BArgs& a, int p, float* xs, int lane) {
-  const int f = a.p[p].fmt;
-  if ((kFmts & fmt_bit(LBQ_TERN5)) && f == LBQ_TERN5) xload_product<LBQ_TERN5>(a, p, xs, lane);
-  if ((kFmts & fmt_bit(LBQ_SIGN1)) && f == LBQ_SIGN1) xload_product<LBQ_SIGN1>(a, p, xs, lane);
-  if ((kFmts & fmt_bit(LBQ_Q2RHT)) && f == LBQ_Q2RHT) xload_product<LBQ_Q2RHT>(a, p, xs, lane);
-}
-
-// Shares of product p this CTA works on (virtual CTAs blockIdx.x, + gridDim.x, ...).
-__device__ __forceinline__ unsigned shares_of(const BArgs& a, int p) {
-  const int participants = a.p[p].KS * a.p[p].G;
-  return static_cast<int>(blockIdx.x) < participants
-             ? static_cast<unsigned>((participants - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1)
-             : 0u;
-}
-
-// The helper readies product p: its x slice, the checks on other CTAs' progress, the L2
-// prefetch of its first units; then opens its gate.
-template <int FMT>
-__device__ __forceinline__ Part first_part(const BProd& P) {
-  return static_cast<int>(blockIdx.x) < P.KS * P.G ? part_of<FMT>(P, blockIdx.x) : Part{0, 0, 0, 1};
-}
-
-template <int kFmts>
-__device__ __forceinline__ bool helper_prepare(const BArgs& a, int p, float* xbuf, volatile Flags* fl,
-                                               Prep* prep, int lane, bool ok) {
-  if (lane == 0) {  // the share and the sum plan, for the compute warps
-    Prep pr;
-    const int f = a.p[p].fmt;
-    pr.pt = (kFmts & fmt_bit(LBQ_TERN5)) && f == LBQ_TERN5   ? first_part<LBQ_TERN5>(a.p[p])
-            : (kFmts & fmt_bit(LBQ_SIGN1)) && f == LBQ_SIGN1 ? first_part<LBQ_SIGN1>(a.p[p])
-                                                             : first_part<LBQ_Q2RHT>(a.p[p]);
-    pr.rp = p - kLag >= 0 ? reduce_plan(a.p[p - kLag]) : RedPlan{0, 0, 0, 1};
-    prep[p % kXBufs] = pr;
-  }
-  // the two counters are read (lane 0) while the x slice loads are in flight
-  const int q = p - kLag;
-  const bool need_done = q >= 0 && a.p[q].KS > 1, need_red = a.p[p].KS > 1 && p >= kRing;
-  const unsigned done_target = need_done ? static_cast<unsigned>(a.p[q].KS * a.p[q].G) : 0u;
-  unsigned dv = 0, rv = 0;
-  if (lane == 0 && need_done) dv = ld_acquire(a.ctr + kCtrDone + q);
-  if (lane == 0 && need_red) rv = ld_acquire(a.ctr + kCtrReduced + (p - kRing));
-  xload_any<kFmts>(a, p, xbuf + (p % kXBufs) * (kXBytes / 4), lane);
-  if (lane == 0 && ok && need_done && dv < done_target)
-    ok = wait_count(a.ctr + kCtrDone + q, done_target, a.fault);
-  if (lane == 0 && ok && need_red && rv < gridDim.x)
-    ok = wait_count(a.ctr + kCtrReduced + (p - kRing), gridDim.x, a.fault);
-  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-  __syncwarp();
-  if (lane == 0) st_release_cta(&fl->gate, p + 1);  // (x slice stores released too)
-#if LBQ_BATCH_HELPER_PREFETCH == 1
-  prefetch_any<kFmts>(a, p + 0, lane);
-#endif
-  return ok;
-}
-
-template <int kFmts>
-__global__ void __maxnreg__(kMaxRegs) gemv_batch_kernel(const __grid_constant__ BArgs a0) {
+__global__ void __launch_bounds__(kThreads, 1) gemv_batch_kernel(const __grid_constant__ BArgs a) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // shared memory: the 128 KB table at the first 64 KB boundary (its page addressing
+  // keeps the base in the upper half of the PRMT operand), the running sums below it
+  // when they fit there, the x staging and the padded x slice above it
   const uint32_t sbase = smem_u32(smem);
   const uint32_t tbase = (sbase + kPage - 1) & ~(kPage - 1);
-  const bool misc_low = tbase - sbase >= kMiscBytes + kDescSmem;
-  const uint32_t misc = misc_low ? sbase : tbase + kTableBytes;
-  float* xbuf = reinterpret_cast<float*>(smem + (misc - sbase));  // two x slices
-  volatile Flags* fl = reinterpret_cast<volatile Flags*>(smem + (misc - sbase) + kXBufs * kXBytes);
-  Prep* prep = reinterpret_cast<Prep*>(smem + (misc - sbase) + kXBufs * kXBytes + 64);
-  // the product list in shared memory (every product start reads its descriptor)
-  const uint32_t dsc = misc + kMiscBytes;  // after the x slices and flags, below or above the table
-  const bool layout_ok = tbase + kTableBytes <= sbase + kSmemBatch && dsc + kDescSmem <= sbase + kSmemBatch &&
-                         (!misc_low || dsc + kDescSmem <= tbase);
-  BProd* dsm = reinterpret_cast<BProd*>(smem + (dsc - sbase));
-  if (layout_ok) {
-    const uint4* src = reinterpret_cast<const uint4*>(a0.p);
-    uint4* dst = reinterpret_cast<uint4*>(dsm);
-    for (int i = tid; i < a0.n * static_cast<int>(sizeof(BProd) / 16); i += blockDim.x) dst[i] = src[i];
-  }
-  if (tid == 0 && layout_ok) {
-    fl->started = 0;
-    fl->built = 0;
-    fl->gate = 0;
-    fl->unitsdone = 0;
-  }
-  __syncthreads();
-  BArgs a = a0;
-  a.p = dsm;
-  if (!layout_ok) {
+  const bool acc_low = tbase - sbase >= kAccBytes;
+  const uint32_t acc = acc_low ? sbase : tbase + kTableBytes;
+  const uint32_t misc = acc_low ? tbase + kTableBytes : acc + kAccBytes;
+  if (tbase + kTableBytes > sbase + kSmemBatch || misc + kMiscBytes > sbase + kSmemBatch) {
     if (tid == 0) atomicExch(a.fault, kFaultBatchLayout);  // cannot happen with a 0 or 1 KB prefix
-    // still count this CTA out, so that the counters end at zero
-  } else if (warp < kCWarps) {
-    bool ok = true;
-    for (int p = 0; p < a.n; ++p) {
-      if (tid == 0) st_release_cta(&fl->started, p + 1);
-      compute_product<kFmts == fmt_bit(LBQ_TERN5)   ? LBQ_TERN5
-                      : kFmts == fmt_bit(LBQ_SIGN1) ? LBQ_SIGN1
-                                                    : LBQ_Q2RHT>(a, p, tbase, xbuf, fl, prep, tid, ok);
-    }
-    reduce_tail(a, fl, tid, ok);
-  } else {
-    // The helper runs two products ahead of the compute warps. For each product p: once
-    // they have started p, it readies p + 2 (x slice into the buffer p - 1 used, which
-    // they are done with; checks on other CTAs; L2 prefetch) and opens its gate; once
-    // they have finished p's units, it releases this CTA's count for p (and for the
-    // sum of p - kLag done with it) at GPU scope, off their path.
-    bool ok = helper_prepare<kFmts>(a, 0, xbuf, fl, prep, lane, true);
-    if (a.n > 1) ok = helper_prepare<kFmts>(a, 1, xbuf, fl, prep, lane, ok);
-    for (int p = 0; p < a.n; ++p) {
-      if (!wait_smem(&fl->started, p + 1, a.fault)) break;
-      // product p + 2's x slice goes where p - 1's was: the compute warps are past it
-      if (p + 2 < a.n) ok = helper_prepare<kFmts>(a, p + 2, xbuf, fl, prep, lane, ok);
-#if LBQ_BATCH_HELPER_PREFETCH == 2
-      // the first units of p + 1 into L2, once the compute warps' prologue of p (whose
-      // loads would queue behind these requests) is over
-      if (p + 1 < a.n && wait_smem(&fl->built, p + 1, a.fault)) prefetch_any<kFmts>(a, p + 1, lane);
-#endif
-      if (!wait_smem(&fl->unitsdone, p + 1, a.fault)) break;
-      if (lane == 0) {
-        const unsigned sh = shares_of(a, p);
-        if (sh) red_release(a.ctr + kCtrDone + p, sh);
-        if (p - kLag >= 0) red_release(a.ctr + kCtrReduced + (p - kLag), 1u);
-      }
-    }
-    // the last products' sums: every CTA must be done with them
-    if (lane == 0) {
-      for (int q = a.n - kLag > 0 ? a.n - kLag : 0; q < a.n && ok; ++q)
-        if (a.p[q].KS > 1) ok = wait_count(a.ctr + kCtrDone + q, static_cast<unsigned>(a.p[q].KS * a.p[q].G), a.fault);
-      st_release_cta(&fl->gate, a.n + 1);
-    }
+    return;
   }
-  // count this CTA out; the last one resets the counters for the next launch
+  const uint32_t xraw = misc, draw = misc + kXRawBytes;
+  float* const xs = reinterpret_cast<float*>(smem + (draw + kDRawBytes - sbase));
+  int* const start = reinterpret_cast<int*>(smem + (draw + kDRawBytes + kXsBytes - sbase));
+
+  // this CTA's range of the list's unit-slices, and the product it starts in
+  const int64_t lo = static_cast<int64_t>(blockIdx.x) * a.W / gridDim.x;
+  const int64_t hi = static_cast<int64_t>(blockIdx.x + 1) * a.W / gridDim.x;
+  if (tid == 0) *start = a.n;
   __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    const unsigned prev = atomicAdd(a.ctr + kCtrExit, 1u);
-    if (prev == gridDim.x - 1) {
-      for (int i = 0; i < a.n; ++i) {
-        a.ctr[kCtrDone + i] = 0;
-        a.ctr[kCtrReduced + i] = 0;
-      }
-      a.ctr[kCtrExit] = 0;
-      __threadfence();
-    }
+  if (tid < a.n) {
+    const int64_t c0 = a.p[tid].c0, c1 = tid + 1 < a.n ? a.p[tid + 1].c0 : a.W;
+    if (c0 <= lo && lo < c1) *start = tid;
   }
+  __syncthreads();
+  Seg g = find_piece(a.p, a.n, *start, 0, lo, hi);
+  if (g.p < 0) return;
+
+  const uint32_t lanereg = tbase | static_cast<uint32_t>(lane * 4);
+  const int rloc = 8 * (lane & 1) + 4 * ((lane >> 1) & 1) + 2 * ((lane >> 2) & 1) + ((lane >> 3) & 1);
+  const uint64_t pol = evict_first_policy();
+  int nb = blocks_in<FMT>(a.p[g.p], g.j);
+  x_fetch<FMT>(a.p[g.p], g.j, nb, xraw, draw, tid);
+  Stream st = make_stream<FMT>(a.p[g.p], g.j, nb, g.c0 + warp, lane, word_offset<FMT>(lane, nb));
+  int32_t nt = g.c1 - g.c0 > warp ? (g.c1 - g.c0 - warp + kWarps - 1) / kWarps : 0;
+  UnitRegs ra, rb;
+  if (nt > 0) load_unit<FMT>(st, 0, lane, pol, ra);
+  if (nt > 1) load_unit<FMT>(st, 1, lane, pol, rb);
+  for (;;) {
+    // the slice's x in place, every warp done with the previous table: build this one
+    x_convert<FMT>(nb, xraw, draw, xs, tid);
+    __syncthreads();
+    build_table<FMT, kThreads>(nb, tbase, xs, tid);
+    __syncthreads();
+    const Seg nx = advance(a.p, a.n, g, lo, hi);
+    int nbx = 0;
+    if (nx.p >= 0) {  // the next slice's x comes in behind the units
+      nbx = blocks_in<FMT>(a.p[nx.p], nx.j);
+      x_fetch<FMT>(a.p[nx.p], nx.j, nbx, xraw, draw, tid);
+    }
+    {
+      const BProd& P = a.p[g.p];
+      const int32_t N = P.N;
+      const bool first = g.j == g.j0, last = g.j == g.j1 - 1;
+      uint16_t* const yp = P.S == 1 ? P.y : nullptr;
+      float* const pp = a.partial + P.poff + static_cast<int64_t>(g.s) * N;
+      const int32_t row0 = g.c0 * kRows + rloc;
+      const bool store_lane = lane < 16;
+      // lane l < 16 keeps the running sum of row rloc of each of the warp's units
+      auto finish = [&](float val, int32_t t) {
+        const int32_t ul = warp + kWarps * t;  // unit within the chunk
+        const int32_t row = row0 + kRows * ul;
+        if (store_lane && row < N) {
+          const uint32_t sa = acc + 4u * static_cast<uint32_t>(kRows * ul + rloc);
+          float v = val;
+          if (!first) {
+            float prev;
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(prev) : "r"(sa));
+            v += prev;
+          }
+          if (!last) {
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(sa), "f"(v) : "memory");
+          } else if (yp) {
+            yp[row] = f32_to_bf16_bits(v);
+          } else {
+            pp[row] = v;
+          }
+        }
+      };
+      // two register buffers, one unit's loads in flight while the other is looked
+      // up; unrolled by two so that they swap without copies
+      for (int32_t t = 0; t < nt; t += 2) {
+        finish(unit_sum<FMT>(ra, lanereg, lane), t);
+        if (t + 2 < nt) load_unit<FMT>(st, t + 2, lane, pol, ra);
+        if (t + 1 >= nt) break;
+        finish(unit_sum<FMT>(rb, lanereg, lane), t + 1);
+        if (t + 3 < nt) load_unit<FMT>(st, t + 3, lane, pol, rb);
+      }
+    }
+    if (nx.p < 0) break;
+    // the next slice's first two units, before its table is built
+    g = nx;
+    nb = nbx;
+    st = make_stream<FMT>(a.p[g.p], g.j, nb, g.c0 + warp, lane, word_offset<FMT>(lane, nb));
+    nt = g.c1 - g.c0 > warp ? (g.c1 - g.c0 - warp + kWarps - 1) / kWarps : 0;
+    if (nt > 0) load_unit<FMT>(st, 0, lane, pol, ra);
+    if (nt > 1) load_unit<FMT>(st, 1, lane, pol, rb);
+  }
+}
+
+// The rows of split products: y = the sum of the S piece sums, in piece order.
+__global__ void piece_sum_kernel(const BProd* list, const float* partial) {
+  const BProd& P = list[blockIdx.y];
+  if (P.S <= 1) return;
+  const int32_t row = static_cast<int32_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (row >= P.N) return;
+  const float* src = partial + P.poff + row;
+  float s = 0.0f;
+  for (int k = 0; k < P.S; ++k) s += src[static_cast<int64_t>(k) * P.N];
+  P.y[row] = f32_to_bf16_bits(s);
 }
 
 int slices_for(int32_t fmt, int64_t K) {
@@ -714,42 +438,80 @@ int slices_for(int32_t fmt, int64_t K) {
   return static_cast<int>((K + per - 1) / per);
 }
 
-}  // namespace
+// The schedule of one launch's list: every product's cost, pieces and piece-sum offset.
+struct Plan {
+  int64_t W = 0;               // unit-slices
+  size_t partial_floats = 0;   // piece sums of split products
+  int32_t max_split_rows = 0;  // the largest N among split products (0: none)
+};
 
-// Floats per partial-sum buffer: the largest KS * N of the list, 256-byte multiple.
-size_t ring_floats_for(const lbq_product* ps, int32_t n) {
-  size_t ring = 0;
-  for (int32_t i = 0; i < n; ++i) {
-    const int KS = slices_for(ps[i].w.fmt, ps[i].w.K);
-    if (KS > 1) {
-      const size_t f = static_cast<size_t>(KS) * static_cast<size_t>(ps[i].w.N);
-      if (f > ring) ring = f;
-    }
-  }
-  return (ring + 63) / 64 * 64;
+// Pieces along K for a product of KS slices: enough that one row-unit of a piece costs
+// at most 1 / kMinUnitsPerTable of a CTA's share W / G.
+int pieces_for(int KS, int64_t W, int G) {
+  const int64_t need = (kMinUnitsPerTable * G * static_cast<int64_t>(KS) + W - 1) / W;
+  return static_cast<int>(need < 1 ? 1 : (need > KS ? KS : need));
 }
 
-// [64 KB counters][kRing partial-sum buffers][the product list]
+Plan plan_list(const lbq_product* ps, int32_t n, int G, BProd* out) {
+  Plan pl;
+  for (int32_t i = 0; i < n; ++i)
+    pl.W += static_cast<int64_t>(slices_for(ps[i].w.fmt, ps[i].w.K)) * ((ps[i].w.N + kRows - 1) / kRows);
+  int64_t c0 = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const lbq_weights& w = ps[i].w;
+    const int KS = slices_for(w.fmt, w.K);
+    const int64_t NU = (w.N + kRows - 1) / kRows;
+    const int S = pieces_for(KS, pl.W, G);
+    if (out) {
+      BProd& P = out[i];
+      P.codes = static_cast<const uint8_t*>(w.codes);
+      P.scales = static_cast<const uint16_t*>(w.scales);
+      P.x = ps[i].x;
+      P.D = ps[i].D;
+      P.y = ps[i].y;
+      P.c0 = c0;
+      P.poff = S > 1 ? static_cast<int64_t>(pl.partial_floats) : 0;
+      P.cstride = static_cast<int32_t>(w.code_stride);
+      P.sstride = static_cast<int32_t>(w.scale_stride);
+      P.N = static_cast<int32_t>(w.N);
+      P.NU = static_cast<int32_t>(NU);
+      P.fmt = static_cast<int16_t>(w.fmt);
+      P.KS = static_cast<int16_t>(KS);
+      P.S = static_cast<int16_t>(S);
+      P.nblk = static_cast<int16_t>(w.K / (w.fmt == LBQ_Q2RHT ? kQ2Block : kTernBlock));
+    }
+    if (S > 1) {
+      pl.partial_floats += static_cast<size_t>(S) * static_cast<size_t>(w.N);
+      if (w.N > pl.max_split_rows) pl.max_split_rows = static_cast<int32_t>(w.N);
+    }
+    c0 += KS * NU;
+  }
+  pl.partial_floats = (pl.partial_floats + 63) / 64 * 64;
+  return pl;
+}
+
+}  // namespace
+
+// [64 KB kept zero (the counter rule of every workspace)][piece sums][the product list]
 size_t lbq_gemv_batch_ws(const lbq_product* ps, int32_t n) {
-  return kWsCounterBytes + kRing * ring_floats_for(ps, n) * sizeof(float) + kDescBytes;
+  const Plan pl = plan_list(ps, n, sm_count(), nullptr);
+  return kWsCounterBytes + pl.partial_floats * sizeof(float) + kDescBytes;
 }
 
 namespace {
 
 // Sets the kernel's shared-memory limit (once per device) and checks that one CTA fits
 // on an SM; the grid is one CTA per SM (the table takes most of the shared memory).
-template <int kFmts>
+template <int FMT>
 cudaError_t batch_grid(int* grid) {
   static PerDevice<int> cache;
   return cache.get(
       [](int, int* g) {
-        cudaError_t r = cudaFuncSetAttribute(gemv_batch_kernel<kFmts>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t r = cudaFuncSetAttribute(gemv_batch_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kSmemBatch));
         if (r != cudaSuccess) return r;
         int per_sm = 0;
-        r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_batch_kernel<kFmts>, kBThreads,
-                                                          kSmemBatch);
+        r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_batch_kernel<FMT>, kThreads, kSmemBatch);
         if (r != cudaSuccess) return r;
         if (per_sm < 1) return cudaErrorLaunchOutOfResources;  // one CTA does not fit an SM
         *g = sm_count();
@@ -758,73 +520,55 @@ cudaError_t batch_grid(int* grid) {
       grid);
 }
 
-template <int kFmts>
-cudaError_t launch_batch(const BArgs& a, int grid, cudaStream_t s) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kBThreads);
-  cfg.dynamicSmemBytes = kSmemBatch;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_batch_kernel<kFmts>, a);
+template <int FMT>
+cudaError_t launch_list(const lbq_product* ps, int32_t n, void* ws, cudaStream_t s) {
+  int grid = 0;
+  cudaError_t e = batch_grid<FMT>(&grid);
+  if (e != cudaSuccess) return e;
+  unsigned* fault = lbq_fault_word();
+  if (!fault) return cudaErrorInvalidDevicePointer;
+  BInstall in;
+  std::vector<BProd> all(static_cast<size_t>(n));
+  const Plan pl = plan_list(ps, n, grid, all.data());
+  BArgs a;
+  a.partial = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsCounterBytes);
+  BProd* list = reinterpret_cast<BProd*>(static_cast<char*>(ws) + kWsCounterBytes +
+                                         pl.partial_floats * sizeof(float));
+  a.p = list;
+  a.fault = fault;
+  a.W = pl.W;
+  a.n = n;
+  a.pad = 0;
+  // the descriptors, in chunks that fit a launch's parameters
+  in.dst = list;
+  for (int32_t i = 0; i < n; i += kInstallChunk) {
+    in.first = i;
+    in.count = n - i < kInstallChunk ? n - i : kInstallChunk;
+    for (int32_t k = 0; k < in.count; ++k) in.p[k] = all[static_cast<size_t>(i + k)];
+    install_kernel<<<1, kInstallChunk, 0, s>>>(in);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  gemv_batch_kernel<FMT><<<grid, kThreads, kSmemBatch, s>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (pl.max_split_rows > 0) {
+    piece_sum_kernel<<<dim3((pl.max_split_rows + 255) / 256, n), 256, 0, s>>>(list, a.partial);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 }  // namespace
 
 cudaError_t lbq_launch_gemv_batch(const lbq_product* ps, int32_t n, void* ws, cudaStream_t s) {
-  int mask = 0;
-  for (int32_t i = 0; i < n; ++i) mask |= fmt_bit(ps[i].w.fmt);
-  int grid = 0;
-  cudaError_t e = mask == fmt_bit(LBQ_TERN5)   ? batch_grid<1>(&grid)
-                  : mask == fmt_bit(LBQ_SIGN1) ? batch_grid<2>(&grid)
-                  : mask == fmt_bit(LBQ_Q2RHT) ? batch_grid<4>(&grid)
-                                               : cudaErrorInvalidValue;  // one format a launch
-  if (e != cudaSuccess) return e;
-  unsigned* fault = lbq_fault_word();
-  if (!fault) return cudaErrorInvalidDevicePointer;
-  const size_t ring_floats = ring_floats_for(ps, n);
-  BArgs a;
-  a.n = n;
-  a.pad = 0;
-  a.ring_floats = static_cast<int64_t>(ring_floats);
-  a.ring = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsCounterBytes);
-  a.ctr = static_cast<unsigned*>(ws);
-  a.fault = fault;
-  BProd* list = reinterpret_cast<BProd*>(static_cast<char*>(ws) + kWsCounterBytes +
-                                         kRing * ring_floats * sizeof(float));
-  a.p = list;
-  BInstall in;
-  in.dst = list;
-  for (int32_t i = 0; i < n; ++i) {
-    const lbq_weights& w = ps[i].w;
-    BProd& P = in.p[i % kInstallChunk];
-    P.codes = static_cast<const uint8_t*>(w.codes);
-    P.scales = static_cast<const uint16_t*>(w.scales);
-    P.x = ps[i].x;
-    P.D = ps[i].D;
-    P.y = ps[i].y;
-    P.cstride = static_cast<int32_t>(w.code_stride);
-    P.sstride = static_cast<int32_t>(w.scale_stride);
-    P.N = static_cast<int32_t>(w.N);
-    P.fmt = static_cast<int16_t>(w.fmt);
-    P.KS = static_cast<int16_t>(slices_for(w.fmt, w.K));
-    const int64_t NU = (w.N + kRows - 1) / kRows;
-    const int64_t per = grid / P.KS > 1 ? grid / P.KS : 1;
-    P.G = static_cast<int16_t>(per < NU ? per : NU);
-    P.nblk = static_cast<int16_t>(w.K / (w.fmt == LBQ_Q2RHT ? kQ2Block : kTernBlock));
-    if (i % kInstallChunk == kInstallChunk - 1 || i == n - 1) {  // a full chunk, or the last
-      in.first = i - i % kInstallChunk;
-      in.count = i % kInstallChunk + 1;
-      install_kernel<<<1, kInstallChunk, 0, s>>>(in);
-      e = cudaGetLastError();
-      if (e != cudaSuccess) return e;
-    }
+  if (n < 1 || n > kMaxBatch) return cudaErrorInvalidValue;
+  for (int32_t i = 1; i < n; ++i)
+    if (ps[i].w.fmt != ps[0].w.fmt) return cudaErrorInvalidValue;  // one format a launch
+  switch (ps[0].w.fmt) {
+    case LBQ_TERN5: return launch_list<LBQ_TERN5>(ps, n, ws, s);
+    case LBQ_SIGN1: return launch_list<LBQ_SIGN1>(ps, n, ws, s);
+    case LBQ_Q2RHT: return launch_list<LBQ_Q2RHT>(ps, n, ws, s);
+    default: return cudaErrorInvalidValue;
   }
-  return mask == fmt_bit(LBQ_TERN5)   ? launch_batch<1>(a, grid, s)
-         : mask == fmt_bit(LBQ_SIGN1) ? launch_batch<2>(a, grid, s)
-                                      : launch_batch<4>(a, grid, s);
 }
