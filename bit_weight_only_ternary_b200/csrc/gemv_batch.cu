@@ -41,13 +41,18 @@ namespace {
 using namespace lbq;
 using namespace lbq::lut;
 
-// 16 warps (four per scheduler) may use 128 registers a thread.
-constexpr int kWarps = 16;
+// 16 warps (four per scheduler) may use 128 registers a thread. (20 warps at 96
+// registers spill and ran 20-35% slower; 12 or 8 warps with three or four unit
+// buffers ran 5-30% slower.)
+#ifndef LBQ_BATCH_WARPS
+#define LBQ_BATCH_WARPS 16
+#endif
+constexpr int kWarps = LBQ_BATCH_WARPS;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kRows = 16;  // rows per unit (four groups of four)
 // Units a chunk keeps running sums for in shared memory (a multiple of kWarps): 63 KB,
 // the room below a 64 KB-aligned table when the dynamic window starts 1 KB in.
-constexpr int32_t kAccUnits = 1008;
+constexpr int32_t kAccUnits = 1008 / kWarps * kWarps;
 constexpr uint32_t kAccBytes = kAccUnits * kRows * 4;
 // The split rule: one row-unit of a piece may cost at most 1 / kMinUnitsPerTable of a
 // CTA's share, so that a table build serves at least that many units.
@@ -307,6 +312,33 @@ __device__ __forceinline__ void load_unit(const Stream& st, int32_t t, int lane,
   }
 }
 
+// Units a warp asks L2 for ahead of its register loads (0: none). Four measured about
+// 7% faster than none in every format; two to eight alike.
+#ifndef LBQ_BATCH_PD
+#define LBQ_BATCH_PD 4
+#endif
+constexpr int kPD = LBQ_BATCH_PD;
+
+__device__ __forceinline__ void prefetch_line(const void* p) {
+  asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
+}
+// L2 prefetch of the warp's unit t: one line request per group (32 lanes x 16 bytes)
+// and the scale runs of the 1-bit and 2-bit formats; only groups that exist.
+template <int FMT>
+__device__ __forceinline__ void prefetch_unit(const Stream& st, int32_t t, int lane) {
+  const uint8_t* w = st.w + static_cast<uint64_t>(t) * st.ustep;
+  const int32_t left = st.ng - (st.g0 + 4 * kWarps * t);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    if (q < left) prefetch_line(w + q * st.gstride);
+  if (FMT != LBQ_TERN5) {
+    const uint8_t* sp = st.s + static_cast<uint64_t>(t) * st.sustep;
+    const int gl = FMT == LBQ_SIGN1 ? 2 * (lane & 1) + ((lane >> 1) & 1) : 2 * (lane & 1);
+    if (gl < left) prefetch_line(sp);
+    if (FMT == LBQ_Q2RHT && gl + 1 < left) prefetch_line(sp + st.sstep);
+  }
+}
+
 // The lane's word offset within a group's slice run (lanes without a word read a
 // neighbour's: their table entries are zero-weight columns).
 template <int FMT>
@@ -359,6 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_batch_kernel(const __grid_co
   UnitRegs ra, rb;
   if (nt > 0) load_unit<FMT>(st, 0, lane, pol, ra);
   if (nt > 1) load_unit<FMT>(st, 1, lane, pol, rb);
+  for (int32_t u = 2; u < 2 + kPD && u < nt; ++u) prefetch_unit<FMT>(st, u, lane);
   for (;;) {
     // the slice's x in place, every warp done with the previous table: build this one
     x_convert<FMT>(nb, xraw, draw, xs, tid);
@@ -400,24 +433,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_batch_kernel(const __grid_co
           }
         }
       };
-      // two register buffers, one unit's loads in flight while the other is looked
-      // up; unrolled by two so that they swap without copies
+      // two register buffers, one unit's loads in flight while the other is looked up
+      // (three or four, with fewer warps to hold them, measured slower); unrolled by
+      // two so that they swap without copies
       for (int32_t t = 0; t < nt; t += 2) {
+        if (kPD > 0 && t + 2 + kPD < nt) prefetch_unit<FMT>(st, t + 2 + kPD, lane);
         finish(unit_sum<FMT>(ra, lanereg, lane), t);
         if (t + 2 < nt) load_unit<FMT>(st, t + 2, lane, pol, ra);
         if (t + 1 >= nt) break;
+        if (kPD > 0 && t + 3 + kPD < nt) prefetch_unit<FMT>(st, t + 3 + kPD, lane);
         finish(unit_sum<FMT>(rb, lanereg, lane), t + 1);
         if (t + 3 < nt) load_unit<FMT>(st, t + 3, lane, pol, rb);
       }
     }
     if (nx.p < 0) break;
-    // the next slice's first two units, before its table is built
+    // the next slice's first two units, before its table is built (and the next few
+    // asked of L2)
     g = nx;
     nb = nbx;
     st = make_stream<FMT>(a.p[g.p], g.j, nb, g.c0 + warp, lane, word_offset<FMT>(lane, nb));
     nt = g.c1 - g.c0 > warp ? (g.c1 - g.c0 - warp + kWarps - 1) / kWarps : 0;
     if (nt > 0) load_unit<FMT>(st, 0, lane, pol, ra);
     if (nt > 1) load_unit<FMT>(st, 1, lane, pol, rb);
+    for (int32_t u = 2; u < 2 + kPD && u < nt; ++u) prefetch_unit<FMT>(st, u, lane);
   }
 }
 
