@@ -31,8 +31,6 @@
 // in by cp.async while the units run, and each warp's first two units of the next
 // slice are loaded before its table is built, so the weight stream runs on through
 // the build.
-#include <vector>
-
 #include "lut.cuh"
 #include "sm100_async.cuh"
 
@@ -67,8 +65,7 @@ constexpr int kMaxBatch = LBQ_BATCH_MAX;
 static_assert(kAccUnits % kWarps == 0, "chunks are whole rounds of units");
 static_assert(kAccBytes <= 63 * 1024, "the sums fit below the table");
 
-// One product as the kernel sees it (80 bytes), written into the workspace by the
-// install kernel before each launch.
+// One product as the kernel sees it (80 bytes).
 struct __align__(16) BProd {
   const uint8_t* codes;
   const uint16_t* scales;
@@ -87,29 +84,18 @@ struct __align__(16) BProd {
   int16_t nblk;     // scale blocks per row
 };
 static_assert(sizeof(BProd) == 80, "descriptor size");
-constexpr int kInstallChunk = 48;  // descriptors per install launch (parameters < 4 KB)
-constexpr size_t kDescBytes = kMaxBatch * sizeof(BProd);
 
-struct BInstall {
-  int32_t first, count;
-  BProd* dst;
-  BProd p[kInstallChunk];
-};
-static_assert(sizeof(BInstall) <= 4096, "install parameters");
-
+// The launch's parameters, the product list included (about 20 KB: kernel parameters
+// may take up to 32 KB since CUDA 12.1), so nothing is copied before the launch.
 struct BArgs {
-  const BProd* p;   // the list (in the workspace)
   float* partial;   // piece sums of split products
   unsigned* fault;
   int64_t W;        // unit-slices of the whole list
   int32_t n;
   int32_t pad;
+  BProd p[kMaxBatch];
 };
-
-__global__ void install_kernel(const __grid_constant__ BInstall in) {
-  const int i = threadIdx.x;
-  if (i < in.count) in.dst[in.first + i] = in.p[i];
-}
+static_assert(sizeof(BArgs) <= 32764, "kernel parameter limit");
 
 // Weight loads: read once, so they neither allocate in L1 nor stay in L2 for long.
 __device__ __forceinline__ uint64_t evict_first_policy() {
@@ -460,12 +446,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_batch_kernel(const __grid_co
 }
 
 // The rows of split products: y = the sum of the S piece sums, in piece order.
-__global__ void piece_sum_kernel(const BProd* list, const float* partial) {
-  const BProd& P = list[blockIdx.y];
+__global__ void piece_sum_kernel(const __grid_constant__ BArgs a) {
+  const BProd& P = a.p[blockIdx.y];
   if (P.S <= 1) return;
   const int32_t row = static_cast<int32_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (row >= P.N) return;
-  const float* src = partial + P.poff + row;
+  const float* src = a.partial + P.poff + row;
   float s = 0.0f;
   for (int k = 0; k < P.S; ++k) s += src[static_cast<int64_t>(k) * P.N];
   P.y[row] = f32_to_bf16_bits(s);
@@ -530,10 +516,10 @@ Plan plan_list(const lbq_product* ps, int32_t n, int G, BProd* out) {
 
 }  // namespace
 
-// [64 KB kept zero (the counter rule of every workspace)][piece sums][the product list]
+// [64 KB kept zero (the counter rule of every workspace)][piece sums]
 size_t lbq_gemv_batch_ws(const lbq_product* ps, int32_t n) {
   const Plan pl = plan_list(ps, n, sm_count(), nullptr);
-  return kWsCounterBytes + pl.partial_floats * sizeof(float) + kDescBytes;
+  return kWsCounterBytes + pl.partial_floats * sizeof(float);
 }
 
 namespace {
@@ -565,33 +551,18 @@ cudaError_t launch_list(const lbq_product* ps, int32_t n, void* ws, cudaStream_t
   if (e != cudaSuccess) return e;
   unsigned* fault = lbq_fault_word();
   if (!fault) return cudaErrorInvalidDevicePointer;
-  BInstall in;
-  std::vector<BProd> all(static_cast<size_t>(n));
-  const Plan pl = plan_list(ps, n, grid, all.data());
-  BArgs a;
+  static thread_local BArgs a;  // 20 KB: off the stack
+  const Plan pl = plan_list(ps, n, grid, a.p);
   a.partial = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsCounterBytes);
-  BProd* list = reinterpret_cast<BProd*>(static_cast<char*>(ws) + kWsCounterBytes +
-                                         pl.partial_floats * sizeof(float));
-  a.p = list;
   a.fault = fault;
   a.W = pl.W;
   a.n = n;
   a.pad = 0;
-  // the descriptors, in chunks that fit a launch's parameters
-  in.dst = list;
-  for (int32_t i = 0; i < n; i += kInstallChunk) {
-    in.first = i;
-    in.count = n - i < kInstallChunk ? n - i : kInstallChunk;
-    for (int32_t k = 0; k < in.count; ++k) in.p[k] = all[static_cast<size_t>(i + k)];
-    install_kernel<<<1, kInstallChunk, 0, s>>>(in);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
   gemv_batch_kernel<FMT><<<grid, kThreads, kSmemBatch, s>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (pl.max_split_rows > 0) {
-    piece_sum_kernel<<<dim3((pl.max_split_rows + 255) / 256, n), 256, 0, s>>>(list, a.partial);
+    piece_sum_kernel<<<dim3((pl.max_split_rows + 255) / 256, n), 256, 0, s>>>(a);
     e = cudaGetLastError();
   }
   return e;

@@ -282,14 +282,25 @@ struct UnitRegs {
 
 // One transpose-reduce stage: c values -> c / 2; the lane keeps the upper half of the
 // row range if its bit d is set, the lower half otherwise, and adds its partner's.
+// (Rows are added two at a time with paired adds where a stage has two or more.)
 template <int C>
 __device__ __forceinline__ void tr_stage(float (&acc)[16], int lane, int d) {
   const bool up = (lane & d) != 0;
+  if (C >= 4) {
 #pragma unroll
-  for (int r = 0; r < C / 2; ++r) {
-    const float send = up ? acc[r] : acc[r + C / 2];
-    const float keep = up ? acc[r + C / 2] : acc[r];
-    acc[r] = keep + __shfl_xor_sync(0xffffffffu, send, d);
+    for (int r = 0; r < C / 2; r += 2) {
+      const float2 lo = make_float2(acc[r], acc[r + 1]), hi = make_float2(acc[r + C / 2], acc[r + C / 2 + 1]);
+      const float2 send = up ? lo : hi, keep = up ? hi : lo;
+      const float2 recv = make_float2(__shfl_xor_sync(0xffffffffu, send.x, d),
+                                      __shfl_xor_sync(0xffffffffu, send.y, d));
+      const float2 sum = __fadd2_rn(keep, recv);
+      acc[r] = sum.x;
+      acc[r + 1] = sum.y;
+    }
+  } else {
+    const float send = up ? acc[0] : acc[1];
+    const float keep = up ? acc[1] : acc[0];
+    acc[0] = keep + __shfl_xor_sync(0xffffffffu, send, d);
   }
 }
 
