@@ -273,6 +273,35 @@ __device__ __forceinline__ Stream make_stream(const BProd& P, int32_t j, int nb,
   return st;
 }
 
+// Refills a buffer with the warp's unit t, group by group as unit_sum frees it (t < 0:
+// nothing left to load).
+template <int FMT>
+struct UnitRefill {
+  const Stream& st;
+  int32_t t;
+  int lane;
+  uint64_t pol;
+  __device__ __forceinline__ void group(int q, UnitRegs& r) const {
+    if (t < 0) return;
+    const int32_t left = st.ng - (st.g0 + 4 * kWarps * t);
+    const uint8_t* w = st.w + static_cast<uint64_t>(t) * st.ustep + q * st.gstride;
+    r.w[q] = q < left ? ldg_stream(w, pol) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  __device__ __forceinline__ void scales(UnitRegs& r) const {
+    if (t < 0) return;
+    const int32_t left = st.ng - (st.g0 + 4 * kWarps * t);
+    const uint8_t* sp = st.s + static_cast<uint64_t>(t) * st.sustep;
+    if (FMT == LBQ_Q2RHT) {
+      const int gl = 2 * (lane & 1);
+      r.s[0] = gl < left ? ldg_stream2(sp, pol) : make_uint2(0u, 0u);
+      r.s[1] = gl + 1 < left ? ldg_stream2(sp + st.sstep, pol) : make_uint2(0u, 0u);
+    } else {
+      const int gl = 2 * (lane & 1) + ((lane >> 1) & 1);
+      r.s[0] = gl < left ? ldg_stream2(sp, pol) : make_uint2(0u, 0u);
+    }
+  }
+};
+
 template <int FMT>
 __device__ __forceinline__ void load_unit(const Stream& st, int32_t t, int lane, uint64_t pol, UnitRegs& r) {
   const uint8_t* w = st.w + static_cast<uint64_t>(t) * st.ustep;
@@ -420,16 +449,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_batch_kernel(const __grid_co
         }
       };
       // two register buffers, one unit's loads in flight while the other is looked up
-      // (three or four, with fewer warps to hold them, measured slower); unrolled by
-      // two so that they swap without copies
+      // (three or four, with fewer warps to hold them, measured slower), each refilled
+      // group by group as its words are looked up; unrolled by two so that they swap
+      // without copies
       for (int32_t t = 0; t < nt; t += 2) {
         if (kPD > 0 && t + 2 + kPD < nt) prefetch_unit<FMT>(st, t + 2 + kPD, lane);
-        finish(unit_sum<FMT>(ra, lanereg, lane), t);
-        if (t + 2 < nt) load_unit<FMT>(st, t + 2, lane, pol, ra);
+        finish(unit_sum<FMT>(ra, lanereg, lane, UnitRefill<FMT>{st, t + 2 < nt ? t + 2 : -1, lane, pol}), t);
         if (t + 1 >= nt) break;
         if (kPD > 0 && t + 3 + kPD < nt) prefetch_unit<FMT>(st, t + 3 + kPD, lane);
-        finish(unit_sum<FMT>(rb, lanereg, lane), t + 1);
-        if (t + 3 < nt) load_unit<FMT>(st, t + 3, lane, pol, rb);
+        finish(unit_sum<FMT>(rb, lanereg, lane, UnitRefill<FMT>{st, t + 3 < nt ? t + 3 : -1, lane, pol}), t + 1);
       }
     }
     if (nx.p < 0) break;

@@ -304,10 +304,20 @@ __device__ __forceinline__ void tr_stage(float (&acc)[16], int lane, int d) {
   }
 }
 
+// A refill that issues nothing (unit_sum's registers are not reused while it runs).
+struct NoRefill {
+  __device__ __forceinline__ void group(int, UnitRegs&) const {}
+  __device__ __forceinline__ void scales(UnitRegs&) const {}
+};
+
 // Lookups, block scales and the reduction of one unit; returns the sum of row
 // 8 b0 + 4 b1 + 2 b2 + b3 of the unit in every lane (b_k = bit k of the lane).
-template <int FMT>
-__device__ __forceinline__ float unit_sum(const UnitRegs& r, uint32_t lanereg, int lane) {
+// refill.group(q, r) may load the next unit's group q into r.w[q] once its words have
+// been looked up, refill.scales(r) its scales once they have been used, so that the
+// next unit's loads start as early as the registers allow.
+template <int FMT, typename Refill = NoRefill>
+__device__ __forceinline__ float unit_sum(UnitRegs& r, uint32_t lanereg, int lane,
+                                          const Refill& refill = Refill()) {
   float acc[16];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -317,6 +327,7 @@ __device__ __forceinline__ float unit_sum(const UnitRegs& r, uint32_t lanereg, i
     acc[4 * q + 1] = p01.y;
     acc[4 * q + 2] = p23.x;
     acc[4 * q + 3] = p23.y;
+    refill.group(q, r);
   }
   tr_stage<16>(acc, lane, 1);
   if (FMT == LBQ_Q2RHT) {  // 2 lanes a block: rows R .. R + 7 (two groups)
@@ -336,6 +347,7 @@ __device__ __forceinline__ float unit_sum(const UnitRegs& r, uint32_t lanereg, i
     acc[0] *= s.x;
     acc[1] *= s.y;
   }
+  refill.scales(r);
   tr_stage<2>(acc, lane, 8);
   return acc[0] + __shfl_xor_sync(0xffffffffu, acc[0], 16);
 }
