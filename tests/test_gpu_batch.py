@@ -1,4 +1,4 @@
-"""lbq_gemv_batch: many independent batch-1 products in one persistent launch.
+"""lbq_gemv_batch: many independent batch-1 products in one launch.
 
 Every product of a list must give what lbq_gemv gives it: codes are the same packed
 bytes, outputs within 2^-8 * sum_k |w_hat x| of the fp64 oracle. Lists mix formats,
@@ -114,6 +114,53 @@ def test_batch_matches_lbq_gemv_and_more_than_one_launch(L, orc):
         lim = torch.from_numpy(TOL * B[0]).cuda()
         assert torch.all((y.double() - ref).abs() <= 2 * lim)
         assert torch.all((y.double() - torch.from_numpy(Y[0]).cuda()).abs() <= lim)
+
+
+def test_batch_schedule_edges(L, orc):
+    """Lists that reach the corners of the schedule: a one-row product alone (a CTA's
+    share is empty on all but one CTA), products of few rows and many K-slices (split
+    along K into up to one piece per slice, added by the second kernel), and such a
+    product beside ordinary ones (split and whole-K products in one launch)."""
+    lists = [
+        [(TERN5, 1, 128)],
+        [(TERN5, 16, 65536)],
+        [(SIGN1, 5, 131072), (Q2RHT, 19, 32768)],
+        [(TERN5, 7168, 5120), (TERN5, 16, 65536), (TERN5, 33, 2560), (TERN5, 3, 640)],
+        [(Q2RHT, 1, 512), (Q2RHT, 4100, 1024), (Q2RHT, 2, 49152)],
+    ]
+    for li, cases in enumerate(lists):
+        prods = _make(L, orc, cases, 3000 + 100 * li)
+        plist = L.ProductList([(p["pw"], p["x"], p["D"], p["y"]) for p in prods])
+        ws = L.workspace_for_batch(plist)
+        for rep in range(2):
+            for p in prods:
+                p["y"].fill_(5.0)
+            L.lbq_gemv_batch(plist, ws)
+            torch.cuda.synchronize()
+            _check(prods, f"list {li} call {rep}")
+        assert not ws[:65536].any(), "counters not left at zero"
+    assert L.lbq_device_fault() == 0
+
+
+def test_batch_many_row_chunks(L, orc):
+    """2.4 million rows of one product (150000 units, about 1014 a CTA): each CTA runs
+    its rows in more than one chunk of running sums. The rows repeat a 1024-row block,
+    so every output must equal its block row's exactly (a row's sum does not depend on
+    where it falls), and the block rows must match the oracle."""
+    Nb, K, reps = 1024, 512, 2344
+    N = Nb * reps
+    Wb = synth.weights(Nb, K, 4242)
+    x = synth.activations(1, K, 4243)
+    pw = L.lbq_pack(TERN5, Wb.cuda().repeat(reps, 1))
+    y = torch.full((N,), 5.0, dtype=torch.bfloat16, device="cuda")
+    L.lbq_gemv_batch(L.ProductList([(pw, x[0].cuda(), None, y)]))
+    torch.cuda.synchronize()
+    codes, scales = orc.pack(TERN5, Wb.numpy())
+    Y, B = orc.gemm(TERN5, codes, scales, K, synth.bf16_bits(x), None, nthreads=NTHREADS)
+    yb = y[:Nb].double().cpu().numpy()
+    assert np.all(np.abs(yb - Y[0]) <= TOL * B[0])
+    assert torch.equal(y.view(reps, Nb), y[:Nb].expand(reps, Nb)), "a repeated row differs"
+    assert L.lbq_device_fault() == 0
 
 
 def test_batch_in_cuda_graph(L, orc):
