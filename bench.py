@@ -42,7 +42,7 @@ METRIC = "packed-weight HBM GB/s (% of peak) & tok/s-equiv, batch-1 27B-shape GE
 WORKLOADS = {
     # name: (format, M, how the pass runs); format 0: a mixed-format layer (product_fmt).
     # "batch": the pass's independent products (each has its own seeded x) through
-    # lbq_gemv_batch, one persistent launch per 256 products; "chained": one lbq_gemv
+    # lbq_gemv_batch, one launch per format and 256 products; "chained": one lbq_gemv
     # call per product in stream order, each allowed to start only as its predecessor
     # finishes (a decoder's order, where a product's x comes from earlier results);
     # "gemm": one lbq_gemm call per product.
@@ -55,7 +55,7 @@ WORKLOADS = {
 # the workloads measured beside the headline in a one-GPU run (plus the tiny GEMV)
 CONFIG_ORDER = ("tern_chained", "sign", "q2", "mixed", "mixed_chained", "gemm8", "gemm32",
                 "gemm512", "gemm4096")
-MODE_TEXT = {"batch": "independent products, one lbq_gemv_batch call per pass (one persistent launch per format)",
+MODE_TEXT = {"batch": "independent products, one lbq_gemv_batch call per pass (one launch per format)",
              "chained": "one lbq_gemv per product, each chained to the previous",
              "gemm": "one lbq_gemm per product"}
 FMT_NAME = {1: "ternary 5 trits/byte + fp16 scale per 128", 2: "1-bit sign + fp16 scale per 128",
@@ -63,12 +63,17 @@ FMT_NAME = {1: "ternary 5 trits/byte + fp16 scale per 128", 2: "1-bit sign + fp1
             0: "mixed: attention (QKV, O) 2-bit + RHT, FFN (gate+up, down) ternary"}
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
-# dram bytes per launch of the dominant kernel from one ncu capture (one 27B layer, the
-# four products, averaged per launch), keyed by the hash of the kernel source it was
-# taken on; reported as null once that source changes.
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture of
+# an 8-layer pass (one launch) scaled by 8 to the 64-layer launch (the traffic grows
+# with the units processed), keyed by workload and by the hash of the kernel sources
+# it was taken on: reported as null once that source changes.
 NCU_TRAFFIC = {
-    # profiles/gemv_tern_1layer_full.md: 72.42 MB read + 256 B written over the 4 launches
-    ("tern", "6a683c1dec9b0cc5"): 18.104e6,
+    # profiles/gemv_batch_tern_8layer_full.md: 603.58 MB read + 3.58 MB written
+    ("tern", "228841dcf7f62628"): 8 * 607.155e6,
+    # profiles/gemv_batch_sign_8layer_full.md: 388.32 MB read + 4.03 MB written
+    ("sign", "228841dcf7f62628"): 8 * 392.350e6,
+    # profiles/gemv_batch_q2_8layer_full.md: 826.73 MB read + 4.58 MB written
+    ("q2", "228841dcf7f62628"): 8 * 831.312e6,
 }
 
 
@@ -336,15 +341,25 @@ class Pass:
                 L.lbq_gemm(p["pw"], p["X"], Dp, p["Y"], self.ws)
 
 
-def launches_per_step(L, prods, mode):
-    """Our kernels per pass: one persistent launch per format and 256 products of it
-    (batch; the small install kernel that copies each launch's list is not counted), or
-    per product the GEMV plus the split-K sum when K spans several slices (chained)."""
+def launches_per_step(L, prods, mode, sms=148):
+    """Our kernels per pass: for lbq_gemv_batch one launch per format and 256 products of
+    it, plus the piece-sum kernel where the library splits a product along K (its rule:
+    pieces = ceil(64 * SMs * slices / total unit-slices of the launch), at most the
+    slices; none for the 64-layer passes); for chained calls, per product the GEMV plus
+    the split-K sum when K spans several slices."""
     if mode == "batch":
         per_fmt = {}
         for p in prods:
-            per_fmt[p["fmt"]] = per_fmt.get(p["fmt"], 0) + 1
-        return sum((c + L.LBQ_BATCH_MAX - 1) // L.LBQ_BATCH_MAX for c in per_fmt.values())
+            per_fmt.setdefault(p["fmt"], []).append(p)
+        n = 0
+        for lst in per_fmt.values():
+            for i in range(0, len(lst), L.LBQ_BATCH_MAX):
+                chunk = lst[i:i + L.LBQ_BATCH_MAX]
+                ks = [-(-p["K"] // (1024 if p["fmt"] == L.LBQ_SIGN1 else 512)) for p in chunk]
+                W = sum(k * -(-p["N"] // 16) for k, p in zip(ks, chunk))
+                split = any(min(k, -(-64 * sms * k // W)) > 1 for k in ks)
+                n += 1 + int(split)
+        return n
     if mode == "chained":
         return sum(1 + (p["K"] > (1024 if p["fmt"] == L.LBQ_SIGN1 else 512)) for p in prods)
     return None  # lbq_gemm: 2 or 3 kernels per product, as the tile planner decides
@@ -455,8 +470,8 @@ def ours(args):
         clocks = clk.summary(tc0, tc1)
         kernel = {"batch": "lbq_gemv_batch", "chained": "lbq_gemv", "gemm": "lbq_gemm"}[mode]
         # The dominant kernel's launch duration inside the timed region: the timed step
-        # divided by the launches of that kernel in it (the persistent batch kernel: one
-        # launch a step; per-product calls: the step over the products).
+        # divided by the launches of that kernel in it (the batch kernel: one launch a
+        # step per format; per-product calls: the step over the products).
         n_launch = launches if mode == "batch" else len(prods)
         roof = roofline(M, algo_bytes, flops, ms_step, n_launch, f"{kernel} ({args.workload})")
         key = kernel_source_hash(BATCH_SOURCES if mode == "batch" else
@@ -610,6 +625,9 @@ def measure_configs(L, synth, store, args, D, stream, torch, dev, barrier, clk, 
         n_launch = launches if mode == "batch" else len(prods)
         kernel = {"batch": "lbq_gemv_batch", "chained": "lbq_gemv", "gemm": "lbq_gemm"}[mode]
         roof = roofline(M, algo_bytes, flops, ms_step, n_launch, f"{kernel} ({name})")
+        src = kernel_source_hash(BATCH_SOURCES if mode == "batch" else
+                                 GEMV_SOURCES if mode == "chained" else GEMM_SOURCES)
+        roof["traffic"] = NCU_TRAFFIC.get((name, src))
         entry = {"workload": workload_string(fmt, M, args.layers, mode), "M": M, "mode": mode,
                  "ms_per_step": round(ms_step, 5), "steps": steps, "warmup": 3,
                  "weight_bytes_per_step": weight_bytes,

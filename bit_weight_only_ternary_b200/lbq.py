@@ -292,8 +292,8 @@ def lbq_gemv_batch_workspace_bytes(plist: ProductList) -> int:
 
 def lbq_gemv_batch(plist: ProductList, workspace=None, stream=None) -> None:
     """Every product of the list (independent batch-1 products, see include/lbq.h), one
-    persistent launch per LBQ_BATCH_MAX products. The workspace's first 64 KB must be
-    zero when it is first used (workspace_for_batch gives such a buffer)."""
+    launch per format present and LBQ_BATCH_MAX products of it. The workspace's first
+    64 KB must be zero when it is first used (workspace_for_batch gives such a buffer)."""
     if workspace is None:
         workspace = workspace_for_batch(plist)
     wsb = workspace.numel() * workspace.element_size()

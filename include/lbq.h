@@ -223,7 +223,7 @@ lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const in
 lbq_status lbq_read_probe(const void* p, size_t bytes, uint32_t* sink, void* stream);
 
 /* Most products one launch of lbq_gemv_batch takes (longer lists, or lists of several
- * formats, run as several). */
+ * formats, run as several launches). */
 #define LBQ_BATCH_MAX 256
 
 /* One batch-1 product of a list: y = W_hat x (W_hat from w; D for LBQ_Q2RHT, else NULL). */
@@ -234,26 +234,26 @@ typedef struct lbq_product {
   uint16_t* y;        /* device bf16 [N]                           */
 } lbq_product;
 
-/* Bytes of workspace lbq_gemv_batch needs for this list (0 on bad arguments). Its
- * first 64 KB hold counters under the same rule as lbq_workspace_bytes: zero when the
- * workspace is first used, zero again after every completed call. */
+/* Bytes of workspace lbq_gemv_batch needs for this list (0 on bad arguments): 64 KB
+ * kept under the counter rule of lbq_workspace_bytes (zero when the workspace is first
+ * used, zero again after every completed call; this call leaves them untouched), then
+ * the piece sums of the products it splits along K (none for lists of many rows). */
 size_t lbq_gemv_batch_workspace_bytes(const lbq_product* ps, int32_t n);
 
-/* n independent batch-1 products, each with the result lbq_gemv gives it, computed by
- * one persistent launch per format present and LBQ_BATCH_MAX products of it ([tern]
- * §1.2, [block] §2.1-2.2, [sign], [rht]: the same lookup arithmetic as lbq_gemv); a
- * list of several formats runs format by format, in list order within a format (the
- * kernel is compiled once per format: one that chose per product ran about twice as
- * slowly, short of registers). One CTA per SM stays
- * resident for the whole list, so no product pays for a launch, a dependency wait or
- * a separate split-K kernel, and the weight stream runs on between products: while
- * the compute warps rebuild their lookup table for a product, a helper warp has the
- * next product's weights fetched into L2 and adds up the previous product's slice
- * sums. The products must be independent: no x or D of the list may overlap any y
- * of the list, and no two y may overlap (checked on the host: LBQ_ERR_ARG). Products
- * may use different formats and shapes. `ps` is host memory, read during the call
- * only. The launch is cooperative (all CTAs resident at once). Workspace as
- * lbq_gemv_batch_workspace_bytes; calls sharing one workspace must not overlap.
+/* n independent batch-1 products, each within the bound lbq_gemv meets (the same
+ * lookup arithmetic: [tern] §1.2, [block] §2.1-2.2, [sign], [rht]; its fp32 sums run
+ * over the K-slices in slice order, so an output may differ from lbq_gemv's inside the
+ * bound), computed by one launch per format present and LBQ_BATCH_MAX products of it,
+ * in list order within a format. The list's products are laid end to end as 16-row
+ * units of full K and cut into one equal range per SM: each CTA computes whole rows,
+ * slice by slice, keeping running sums in shared memory, and no CTA waits for
+ * another. A product too short in rows for that cut is split along K; its pieces'
+ * fp32 sums go to the workspace and a second kernel adds them in piece order. Results
+ * are deterministic. The products must be independent: no x or D of the list may
+ * overlap any y of the list, and no two y may overlap (checked on the host:
+ * LBQ_ERR_ARG). Products may use different formats and shapes. `ps` is host memory,
+ * read during the call only (the list travels in the launch's parameters). Workspace
+ * as lbq_gemv_batch_workspace_bytes; calls sharing one workspace must not overlap.
  * Errors: those of lbq_gemv for any product, LBQ_ERR_ARG (ps NULL, n < 1, overlap),
  * LBQ_ERR_WORKSPACE, LBQ_ERR_CUDA. */
 lbq_status lbq_gemv_batch(const lbq_product* ps, int32_t n, void* workspace,
@@ -267,7 +267,7 @@ lbq_status lbq_gemv_batch(const lbq_product* ps, int32_t n, void* workspace,
  * kernels (on an mbarrier, for a TMA copy or a slot) is bounded by about 2 s; a
  * wait that runs out records a non-zero *code (3: shared-memory layout of the
  * batch-1 product, 4-9: tensor-core product stages, 10: the batch-1 product's
- * weight copies, 11: lbq_selftest_wait, 12: lbq_gemv_batch's waits on other CTAs,
+ * weight copies, 11: lbq_selftest_wait, 12: unused (lbq_gemv_batch has no waits),
  * 13: lbq_gemv_batch's shared-memory layout) and the kernel returns early with
  * incomplete outputs instead of hanging. Synchronises the device.
  * Returns LBQ_OK with *code = 0 when no wait gave up, LBQ_ERR_DEVICE_WAIT with the
