@@ -87,12 +87,14 @@ static_assert(sizeof(BProd) == 80, "descriptor size");
 
 // The launch's parameters, the product list included (about 20 KB: kernel parameters
 // may take up to 32 KB since CUDA 12.1), so nothing is copied before the launch.
+constexpr int kMaxGrid = 192;  // CTAs a launch may use (one per SM)
 struct BArgs {
   float* partial;   // piece sums of split products
   unsigned* fault;
   int64_t W;        // unit-slices of the whole list
   int32_t n;
   int32_t pad;
+  int64_t bound[kMaxGrid + 1];  // CTA c's range of unit-slices: [bound[c], bound[c + 1])
   BProd p[kMaxBatch];
 };
 static_assert(sizeof(BArgs) <= 32764, "kernel parameter limit");
@@ -340,14 +342,15 @@ __device__ __forceinline__ void prefetch_line(const void* p) {
 // L2 prefetch of the warp's unit t: one line request per group (32 lanes x 16 bytes)
 // and the scale runs of the 1-bit and 2-bit formats; only groups that exist.
 template <int FMT>
-__device__ __forceinline__ void prefetch_unit(const Stream& st, int32_t t, int lane) {
-  const uint8_t* w = st.w + static_cast<uint64_t>(t) * st.ustep;
+__device__ __forceinline__ void prefetch_unit(const Stream& st, int32_t t, int lane, uint32_t dw = 0,
+                                              uint32_t ds = 0) {
+  const uint8_t* w = st.w + static_cast<uint64_t>(t) * st.ustep + dw;
   const int32_t left = st.ng - (st.g0 + 4 * kWarps * t);
 #pragma unroll
   for (int q = 0; q < 4; ++q)
     if (q < left) prefetch_line(w + q * st.gstride);
   if (FMT != LBQ_TERN5) {
-    const uint8_t* sp = st.s + static_cast<uint64_t>(t) * st.sustep;
+    const uint8_t* sp = st.s + static_cast<uint64_t>(t) * st.sustep + ds;
     const int gl = FMT == LBQ_SIGN1 ? 2 * (lane & 1) + ((lane >> 1) & 1) : 2 * (lane & 1);
     if (gl < left) prefetch_line(sp);
     if (FMT == LBQ_Q2RHT && gl + 1 < left) prefetch_line(sp + st.sstep);
@@ -384,8 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_batch_kernel(const __grid_co
   int* const start = reinterpret_cast<int*>(smem + (draw + kDRawBytes + kXsBytes - sbase));
 
   // this CTA's range of the list's unit-slices, and the product it starts in
-  const int64_t lo = static_cast<int64_t>(blockIdx.x) * a.W / gridDim.x;
-  const int64_t hi = static_cast<int64_t>(blockIdx.x + 1) * a.W / gridDim.x;
+  const int64_t lo = a.bound[blockIdx.x], hi = a.bound[blockIdx.x + 1];
   if (tid == 0) *start = a.n;
   __syncthreads();
   if (tid < a.n) {
@@ -419,6 +421,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_batch_kernel(const __grid_co
       nbx = blocks_in<FMT>(a.p[nx.p], nx.j);
       x_fetch<FMT>(a.p[nx.p], nx.j, nbx, xraw, draw, tid);
     }
+    // When the next step is the next slice of the same units (and both slices are
+    // whole), the last units of this slice ask L2 for the first ones of the next: the
+    // same units, one slice further (codes one group run, scales one scale run), so the
+    // stream does not restart cold after the next table build.
+    // (Not for the 2-bit format, measured 3% slower with it: its stream is the closest
+    // to the HBM rate, and the early requests compete with the slice's own.)
+    const bool pf_next = FMT != LBQ_Q2RHT && nx.p == g.p && nx.s == g.s && nx.c0 == g.c0 &&
+                         nx.j == g.j + 1 && nb == Traits<FMT>::kBlocks && nbx == Traits<FMT>::kBlocks;
     {
       const BProd& P = a.p[g.p];
       const int32_t N = P.N;
@@ -448,15 +458,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_batch_kernel(const __grid_co
           }
         }
       };
+      auto prefetch_ahead = [&](int32_t u) {
+        if (u < nt) prefetch_unit<FMT>(st, u, lane);
+        else if (pf_next && u - nt < nt)
+          prefetch_unit<FMT>(st, u - nt, lane, Traits<FMT>::kGroupBytes,
+                             FMT == LBQ_TERN5 ? Traits<FMT>::kGroupBytes : Traits<FMT>::kScaleBytes);
+      };
       // two register buffers, one unit's loads in flight while the other is looked up
       // (three or four, with fewer warps to hold them, measured slower), each refilled
       // group by group as its words are looked up; unrolled by two so that they swap
       // without copies
       for (int32_t t = 0; t < nt; t += 2) {
-        if (kPD > 0 && t + 2 + kPD < nt) prefetch_unit<FMT>(st, t + 2 + kPD, lane);
+        if (kPD > 0) prefetch_ahead(t + 2 + kPD);
         finish(unit_sum<FMT>(ra, lanereg, lane, UnitRefill<FMT>{st, t + 2 < nt ? t + 2 : -1, lane, pol}), t);
         if (t + 1 >= nt) break;
-        if (kPD > 0 && t + 3 + kPD < nt) prefetch_unit<FMT>(st, t + 3 + kPD, lane);
+        if (kPD > 0) prefetch_ahead(t + 3 + kPD);
         finish(unit_sum<FMT>(rb, lanereg, lane, UnitRefill<FMT>{st, t + 3 < nt ? t + 3 : -1, lane, pol}), t + 1);
       }
     }
@@ -542,6 +558,74 @@ Plan plan_list(const lbq_product* ps, int32_t n, int G, BProd* out) {
   return pl;
 }
 
+// A table build (with the stream's restart behind it) costs about as much time as this
+// many unit-slices (measured: ternary CTAs ended 4.2 us later per build, at 0.077 us a
+// unit-slice, before the next slice's first units were prefetched across the build;
+// 32 and 54 measured alike after it, 0 about 3% slower).
+#ifndef LBQ_BATCH_BUILD_COST
+#define LBQ_BATCH_BUILD_COST 48
+#endif
+constexpr int64_t kBuildCost = LBQ_BATCH_BUILD_COST;
+
+// One greedy pass of the cut for a target cost T per CTA: each CTA takes the list's
+// next units in order while its cost (unit-slices plus kBuildCost per table it will
+// build: every chunk of every piece builds one table per slice of the piece) stays
+// within T. Fills bound[0..G] (the first unit-slice of each CTA's range; W past the
+// last) and returns whether every unit found a CTA.
+bool cut_for(const BProd* P, int32_t n, int G, int64_t W, int64_t T, int64_t* bound) {
+  int32_t p = 0, s = 0;
+  int64_t u = 0;  // the next unassigned unit of piece s of product p
+  auto skip_done = [&]() {
+    while (p < n && u >= P[p].NU) {
+      u = 0;
+      if (++s >= P[p].S) { s = 0; ++p; }
+    }
+  };
+  skip_done();
+  for (int c = 0; c < G; ++c) {
+    if (p >= n) { bound[c] = W; continue; }
+    const int32_t j0 = static_cast<int32_t>(static_cast<int64_t>(P[p].KS) * s / P[p].S);
+    bound[c] = P[p].c0 + static_cast<int64_t>(P[p].NU) * j0 + u * (static_cast<int64_t>(P[p].KS) * (s + 1) / P[p].S - j0);
+    int64_t cost = 0;
+    while (p < n) {
+      const int64_t a = static_cast<int64_t>(P[p].KS) * s / P[p].S;
+      const int64_t len = static_cast<int64_t>(P[p].KS) * (s + 1) / P[p].S - a;
+      // chunks of this CTA's units of the piece, from its first one
+      int64_t in_piece = 0;
+      bool stop = false;
+      while (u < P[p].NU) {
+        const int64_t chunk_room = kAccUnits - in_piece % kAccUnits;
+        const int64_t start_cost = in_piece % kAccUnits == 0 ? kBuildCost * len : 0;
+        const int64_t afford = (T - cost - start_cost) / len;
+        if (afford <= 0) { stop = true; break; }
+        int64_t k = afford < chunk_room ? afford : chunk_room;
+        if (k > P[p].NU - u) k = P[p].NU - u;
+        cost += start_cost + k * len;
+        u += k;
+        in_piece += k;
+        if (k < chunk_room && u < P[p].NU) { stop = true; break; }
+      }
+      if (stop) break;
+      skip_done();
+    }
+  }
+  bound[G] = W;
+  return p >= n;
+}
+
+// The cut with the smallest T that places every unit (bisection; each pass is linear
+// in the CTAs and the list's chunks).
+void plan_cut(const BProd* P, int32_t n, int G, int64_t W, int64_t* bound) {
+  int64_t lo = (W + G - 1) / G, hi = lo;
+  while (!cut_for(P, n, G, W, hi, bound)) hi *= 2;
+  while (lo < hi) {
+    const int64_t mid = lo + (hi - lo) / 2;
+    if (cut_for(P, n, G, W, mid, bound)) hi = mid;
+    else lo = mid + 1;
+  }
+  cut_for(P, n, G, W, hi, bound);
+}
+
 }  // namespace
 
 // [64 KB kept zero (the counter rule of every workspace)][piece sums]
@@ -566,7 +650,7 @@ cudaError_t batch_grid(int* grid) {
         r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_batch_kernel<FMT>, kThreads, kSmemBatch);
         if (r != cudaSuccess) return r;
         if (per_sm < 1) return cudaErrorLaunchOutOfResources;  // one CTA does not fit an SM
-        *g = sm_count();
+        *g = sm_count() < kMaxGrid ? sm_count() : kMaxGrid;
         return cudaSuccess;
       },
       grid);
@@ -586,6 +670,7 @@ cudaError_t launch_list(const lbq_product* ps, int32_t n, void* ws, cudaStream_t
   a.W = pl.W;
   a.n = n;
   a.pad = 0;
+  plan_cut(a.p, n, grid, pl.W, a.bound);
   gemv_batch_kernel<FMT><<<grid, kThreads, kSmemBatch, s>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
