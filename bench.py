@@ -68,12 +68,12 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 # with the units processed), keyed by workload and by the hash of the kernel sources
 # it was taken on: reported as null once that source changes.
 NCU_TRAFFIC = {
-    # profiles/gemv_batch_tern_8layer_full.md: 603.58 MB read + 3.58 MB written
-    ("tern", "228841dcf7f62628"): 8 * 607.155e6,
-    # profiles/gemv_batch_sign_8layer_full.md: 388.32 MB read + 4.03 MB written
-    ("sign", "228841dcf7f62628"): 8 * 392.350e6,
-    # profiles/gemv_batch_q2_8layer_full.md: 826.73 MB read + 4.58 MB written
-    ("q2", "228841dcf7f62628"): 8 * 831.312e6,
+    # profiles/gemv_batch_tern_8layer_full.md: 605.54 MB read + 3.60 MB written
+    ("tern", "ddad2f6d44495dbb"): 8 * 609.143e6,
+    # profiles/gemv_batch_sign_8layer_full.md: 388.97 MB read + 5.70 MB written
+    ("sign", "ddad2f6d44495dbb"): 8 * 394.667e6,
+    # profiles/gemv_batch_q2_8layer_full.md: 826.45 MB read + 3.56 MB written
+    ("q2", "ddad2f6d44495dbb"): 8 * 830.004e6,
 }
 
 
