@@ -9,8 +9,10 @@
 // Work is counted in unit-slices: one 16-row unit of one K-slice (512 weights; 1024 for
 // the 1-bit format). A product of KS slices and NU units costs KS * NU. The list's
 // products are laid end to end, each as NU row-units of full K, and the total is cut
-// into one equal, contiguous range per CTA (one CTA per SM): every CTA computes whole
-// rows of one or a few products, all of K, so its rows need nobody else's sums. It
+// into one contiguous range per CTA (one CTA per SM), the ranges of equal cost: their
+// unit-slices plus a fixed charge per table the range will build (plan_cut, on the
+// host). Every CTA computes whole rows of one or a few products, all of K, so its rows
+// need nobody else's sums. It
 // walks its range slice by slice: for each slice it builds the 128 KB lookup table of
 // that slice of x once and runs all its units of that product through it, keeping
 // each row's running sum in shared memory (in chunks of up to kAccUnits units), so a
@@ -28,9 +30,9 @@
 // lane loads its word of four rows per group with 16-byte global loads (no L1
 // allocation, evict-first in L2), one unit ahead, looks its bytes up, and the warp
 // reduces the unit's 16 rows with the butterfly of lut.cuh. The next slice's x comes
-// in by cp.async while the units run, and each warp's first two units of the next
-// slice are loaded before its table is built, so the weight stream runs on through
-// the build.
+// in by cp.async while the units run; the last units of a slice ask L2 for the first
+// ones of the next, and each warp's first two units of the next slice are loaded before
+// its table is built, so the weight stream runs on through the build.
 #include "lut.cuh"
 #include "sm100_async.cuh"
 

@@ -245,7 +245,8 @@ size_t lbq_gemv_batch_workspace_bytes(const lbq_product* ps, int32_t n);
  * over the K-slices in slice order, so an output may differ from lbq_gemv's inside the
  * bound), computed by one launch per format present and LBQ_BATCH_MAX products of it,
  * in list order within a format. The list's products are laid end to end as 16-row
- * units of full K and cut into one equal range per SM: each CTA computes whole rows,
+ * units of full K and cut into one range per SM, of equal cost (units plus table
+ * builds): each CTA computes whole rows,
  * slice by slice, keeping running sums in shared memory, and no CTA waits for
  * another. A product too short in rows for that cut is split along K; its pieces'
  * fp32 sums go to the workspace and a second kernel adds them in piece order. Results
