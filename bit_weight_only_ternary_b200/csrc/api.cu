@@ -305,6 +305,18 @@ lbq_status lbq_gemv_batch(const lbq_product* ps, int32_t n, void* workspace,
   return st;
 }
 
+lbq_status lbq_gemv_batch_plan(const lbq_product* ps, int32_t n, int32_t ctas, int32_t* pieces,
+                               int64_t* bound, int64_t* total) {
+  if (!pieces || !bound || !total || ctas < 1 || ctas > LBQ_BATCH_MAX_CTAS || n > LBQ_BATCH_MAX)
+    return LBQ_ERR_ARG;
+  const lbq_status st = check_batch(ps, n);
+  if (st != LBQ_OK) return st;
+  for (int32_t i = 1; i < n; ++i)
+    if (ps[i].w.fmt != ps[0].w.fmt) return LBQ_ERR_ARG;
+  *total = lbq_gemv_batch_plan_list(ps, n, ctas, pieces, bound);
+  return LBQ_OK;
+}
+
 lbq_status lbq_gemm(const lbq_weights* w, const uint16_t* X, int64_t M, const int8_t* D,
                     uint16_t* Y, void* workspace, size_t workspace_bytes, void* stream) {
   Layout L;

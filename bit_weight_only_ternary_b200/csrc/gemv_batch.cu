@@ -33,6 +33,8 @@
 // in by cp.async while the units run; the last units of a slice ask L2 for the first
 // ones of the next, and each warp's first two units of the next slice are loaded before
 // its table is built, so the weight stream runs on through the build.
+#include <vector>
+
 #include "lut.cuh"
 #include "sm100_async.cuh"
 
@@ -89,7 +91,7 @@ static_assert(sizeof(BProd) == 80, "descriptor size");
 
 // The launch's parameters, the product list included (about 20 KB: kernel parameters
 // may take up to 32 KB since CUDA 12.1), so nothing is copied before the launch.
-constexpr int kMaxGrid = 192;  // CTAs a launch may use (one per SM)
+constexpr int kMaxGrid = LBQ_BATCH_MAX_CTAS;  // CTAs a launch may use (one per SM)
 struct BArgs {
   float* partial;   // piece sums of split products
   unsigned* fault;
@@ -629,6 +631,17 @@ void plan_cut(const BProd* P, int32_t n, int G, int64_t W, int64_t* bound) {
 }
 
 }  // namespace
+
+// The schedule of one launch's list for `ctas` CTAs (host only): pieces per product and
+// the CTAs' boundaries, exactly as launch_list computes them.
+int64_t lbq_gemv_batch_plan_list(const lbq_product* ps, int32_t n, int ctas, int32_t* pieces,
+                                 int64_t* bound) {
+  std::vector<BProd> all(static_cast<size_t>(n));
+  const Plan pl = plan_list(ps, n, ctas, all.data());
+  for (int32_t i = 0; i < n; ++i) pieces[i] = all[static_cast<size_t>(i)].S;
+  plan_cut(all.data(), n, ctas, pl.W, bound);
+  return pl.W;
+}
 
 // [64 KB kept zero (the counter rule of every workspace)][piece sums]
 size_t lbq_gemv_batch_ws(const lbq_product* ps, int32_t n) {

@@ -170,6 +170,8 @@ size_t lbq_gemm_workspace(const lbq_weights* w, int64_t M);
 // The batched batch-1 products (gemv_batch.cu): workspace for a list of at most
 // LBQ_BATCH_MAX products, and one launch over such a list.
 size_t lbq_gemv_batch_ws(const lbq_product* ps, int32_t n);
+int64_t lbq_gemv_batch_plan_list(const lbq_product* ps, int32_t n, int ctas, int32_t* pieces,
+                                 int64_t* bound);
 cudaError_t lbq_launch_gemv_batch(const lbq_product* ps, int32_t n, void* ws, cudaStream_t s);
 size_t lbq_gemm_tc_workspace(const lbq_weights* w, int64_t M);
 cudaError_t lbq_launch_gemm_tc(const lbq_weights* w, const uint16_t* X, int64_t M, uint16_t* Y,

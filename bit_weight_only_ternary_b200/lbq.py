@@ -23,8 +23,9 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblbq.so")
 EXPORTS = ("lbq_status_string", "lbq_packed_layout", "lbq_pack", "lbq_unpack", "lbq_rht_signs",
            "lbq_hadamard", "lbq_workspace_bytes", "lbq_gemv", "lbq_gemm", "lbq_gemv_noalloc", "lbq_device_fault",
            "lbq_selftest_wait", "lbq_read_probe", "lbq_gemv_batch_workspace_bytes", "lbq_gemv_batch",
-           "lbq_last_cuda_error", "lbq_last_cuda_error_string", "lbq_gemv_f32")
+           "lbq_last_cuda_error", "lbq_last_cuda_error_string", "lbq_gemv_f32", "lbq_gemv_batch_plan")
 LBQ_BATCH_MAX = 256
+LBQ_BATCH_MAX_CTAS = 192
 LBQ_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -72,6 +73,7 @@ def _load():
         "lbq_read_probe": (ctypes.c_int, [p, sz, p, p]),
         "lbq_gemv_batch_workspace_bytes": (sz, [ctypes.POINTER(lbq_product), i32]),
         "lbq_gemv_batch": (ctypes.c_int, [ctypes.POINTER(lbq_product), i32, p, sz, p]),
+        "lbq_gemv_batch_plan": (ctypes.c_int, [ctypes.POINTER(lbq_product), i32, i32, p, p, p]),
         "lbq_last_cuda_error": (i32, []),
         "lbq_last_cuda_error_string": (ctypes.c_char_p, []),
     }
@@ -284,6 +286,18 @@ class ProductList:
 
     def __len__(self):
         return len(self.items)
+
+
+def lbq_gemv_batch_plan(arr, n: int, ctas: int):
+    """The schedule one launch of lbq_gemv_batch gives a list of one format (host only):
+    (pieces per product, CTA boundaries [ctas + 1], total unit-slices). `arr` is a
+    ctypes array of lbq_product (ProductList.arr, or records built by hand)."""
+    pieces = (ctypes.c_int32 * n)()
+    bound = (ctypes.c_int64 * (ctas + 1))()
+    total = ctypes.c_int64()
+    _check(_lib.lbq_gemv_batch_plan(arr, n, ctas, pieces, bound, ctypes.byref(total)),
+           "lbq_gemv_batch_plan")
+    return list(pieces), list(bound), int(total.value)
 
 
 def lbq_gemv_batch_workspace_bytes(plist: ProductList) -> int:

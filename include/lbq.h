@@ -260,6 +260,24 @@ size_t lbq_gemv_batch_workspace_bytes(const lbq_product* ps, int32_t n);
 lbq_status lbq_gemv_batch(const lbq_product* ps, int32_t n, void* workspace,
                           size_t workspace_bytes, void* stream);
 
+/* Most CTAs one launch of lbq_gemv_batch uses (one per SM, at most this many). */
+#define LBQ_BATCH_MAX_CTAS 192
+
+/* The schedule lbq_gemv_batch gives one launch's list when it runs `ctas` CTAs (it runs
+ * one per SM): host only, no device work, for inspection and tests. The list must be
+ * one launch's: one format, 1..LBQ_BATCH_MAX products, valid as for lbq_gemv_batch.
+ * Work is counted in unit-slices (one 16-row unit of one K-slice: 512 weights, 1024 for
+ * LBQ_SIGN1); product i has KS_i slices, NU_i = ceil(N_i / 16) units and starts at
+ * c0_i = sum of KS_j * NU_j over j < i. Writes pieces[i] (host int32 [n]): the pieces
+ * product i is split into along K (piece s holds slices [KS s / S, KS (s + 1) / S); 1:
+ * whole rows on one CTA), bound (host int64 [ctas + 1]): CTA c computes the units
+ * whose first unit-slice lies in [bound[c], bound[c + 1]) (unit u of piece s of product
+ * i starts at c0_i + NU_i * j0 + u * (j1 - j0)), and *total, the list's unit-slices.
+ * Errors: LBQ_ERR_ARG (NULL outputs, ctas < 1 or > LBQ_BATCH_MAX_CTAS, n > LBQ_BATCH_MAX,
+ * mixed formats), and those of lbq_gemv_batch's checks. */
+lbq_status lbq_gemv_batch_plan(const lbq_product* ps, int32_t n, int32_t ctas, int32_t* pieces,
+                               int64_t* bound, int64_t* total);
+
 /* Size of the scratch array that lbq_gemv_noalloc uses (4 MiB). */
 #define LBQ_NOALLOC_SCRATCH_BYTES (4u << 20)
 
