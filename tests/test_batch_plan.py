@@ -153,3 +153,25 @@ def test_plan_rejects_bad_arguments(L):
     pieces = (ctypes.c_int32 * 1)()
     total = ctypes.c_int64()
     assert L._lib.lbq_gemv_batch_plan(one, 1, 148, pieces, None, ctypes.byref(total)) == L.LBQ_ERR_ARG
+
+
+def test_bench_counts_the_launches_the_library_makes(L):
+    """bench.py claims its kernel launches from the library's split rule; that rule must
+    agree with the plan (a launch adds the piece-sum kernel when any product splits)."""
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    rng = random.Random(5)
+    lists = [[(TERN5, K, N) for K, N in LAYER], [(TERN5, K, N) for _ in range(64) for K, N in LAYER],
+             [(SIGN1, 131072, 5)], [(Q2RHT, 1024, 4100)]]
+    for _ in range(10):
+        fmt = rng.choice([TERN5, SIGN1, Q2RHT])
+        lists.append([(fmt, 512 * rng.randint(1, 12) if fmt == Q2RHT else 128 * rng.randint(1, 40),
+                       rng.randint(1, 6000)) for _ in range(rng.randint(1, 30))])
+    for cases in lists:
+        for i in range(0, len(cases), L.LBQ_BATCH_MAX):
+            chunk = cases[i:i + L.LBQ_BATCH_MAX]
+            pieces, _, _ = L.lbq_gemv_batch_plan(records(L, chunk), len(chunk), 148)
+            prods = [dict(fmt=f, K=K, N=N) for f, K, N in chunk]
+            assert bench.launches_per_step(L, prods, "batch") == 1 + int(max(pieces) > 1)
